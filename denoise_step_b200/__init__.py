@@ -1,0 +1,302 @@
+"""denoise_step_b200: the streaming pyramid denoising round on B200 (sm_100a).
+
+A thin ctypes binding over the C ABI in include/pl.h (libpl.so, built in-tree
+by `python -m denoise_step_b200.build`). Every step of the round runs in the
+library's CUDA kernels; this module only marshals arguments (torch tensors
+supply device memory and streams). There is no CPU fallback: importing the
+package without the built library raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libpl.so")
+
+PL_OK, PL_EINVAL, PL_ESTATE, PL_ENOMEM, PL_ECUDA, PL_ETIMEOUT, PL_EDEVICE, PL_EUNSUPPORTED = range(8)
+MAX_LAYERS = 16
+
+
+class PLError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib.pl_status_string(status).decode()} (status {status})")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m denoise_step_b200.build`")
+lib = C.CDLL(LIB_PATH)
+
+vp, i32, i64, f32, sz = C.c_void_p, C.c_int, C.c_int64, C.c_float, C.c_size_t
+
+
+class KVSegment(C.Structure):
+    _fields_ = [("k", vp), ("v", vp), ("len", i64), ("ld", i64), ("frame_stride", i64)]
+
+
+class Config(C.Structure):
+    _fields_ = [("latent_c", C.c_int32), ("latent_h", C.c_int32), ("latent_w", C.c_int32),
+                ("n_layers", C.c_int32), ("layer_tokens", C.c_int32 * MAX_LAYERS),
+                ("layer_channels", C.c_int32 * MAX_LAYERS), ("heads", C.c_int32),
+                ("drift_threshold", C.c_float), ("append_cap", C.c_int32)]
+
+
+class LayerWeights(C.Structure):
+    _fields_ = [("w_qkv", vp), ("w_o", vp), ("m_q", vp), ("m_kv", vp), ("m_o", vp)]
+
+
+class State(C.Structure):
+    _fields_ = [("initialised", C.c_int32), ("head", C.c_int32), ("slot_t", C.c_int32 * 4),
+                ("rounds", C.c_int64), ("frames_in", C.c_int64), ("frames_out", C.c_int64),
+                ("bank_count", C.c_int32), ("appends", C.c_int32), ("device_status", C.c_uint32)]
+
+    def as_dict(self):
+        return {"initialised": self.initialised, "head": self.head, "slot_t": list(self.slot_t),
+                "rounds": self.rounds, "frames_in": self.frames_in, "frames_out": self.frames_out,
+                "bank_count": self.bank_count, "appends": self.appends,
+                "device_status": self.device_status}
+
+
+_SIGS = {
+    "pl_status_string": (C.c_char_p, [i32]),
+    "pl_abi_version": (i32, []),
+    "pl_gemm_f16": (i32, [vp, i64, vp, i64, vp, i64, i32, i32, i32, vp]),
+    "pl_segment_attention": (i32, [vp, i64, i64, C.POINTER(KVSegment), i32, i32, i32, i32, i32,
+                                   vp, i64, i64, vp]),
+    "pl_ref_attention_workspace_bytes": (i32, [i32, i32, i32, i32, C.POINTER(sz)]),
+    "pl_ref_attention": (i32, [vp, vp, vp, C.POINTER(vp), i32, i32, i32, i32, i32, vp, vp, sz, vp]),
+    "pl_motion_xattn_workspace_bytes": (i32, [i32, i32, i32, C.POINTER(sz)]),
+    "pl_motion_xattn": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),
+    "pl_motion_bank_check": (i32, [vp, vp, vp, i32, i32, vp, i32, f32, i32, vp, vp, vp, vp]),
+    "pl_workspace_bytes": (i32, [C.POINTER(Config), C.POINTER(sz)]),
+    "pl_ctx_create": (i32, [C.POINTER(Config), vp, sz, C.POINTER(vp)]),
+    "pl_ctx_destroy": (i32, [vp]),
+    "pl_bank_init": (i32, [vp, C.POINTER(LayerWeights), C.POINTER(vp), C.POINTER(vp), vp, vp, vp,
+                           vp, vp]),
+    "pl_ring_push": (i32, [vp, vp, vp, vp]),
+    "pl_pyramid_ddim_step": (i32, [vp, vp, vp, vp]),
+    "pl_ctx_bank_check": (i32, [vp, vp, i32, vp, vp, vp, vp]),
+    "pl_stream_round": (i32, [vp, vp, vp, C.POINTER(vp), vp, vp, vp, C.POINTER(vp), vp]),
+    "pl_get_state": (i32, [vp, C.POINTER(State), vp]),
+    "pl_get_motion_bank": (i32, [vp, vp, C.POINTER(C.c_int32), vp]),
+    "pl_get_device_status": (i32, [vp, vp]),
+    "pl_ctx_ring_latents": (vp, [vp]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+def check(status: int, what: str) -> None:
+    if status != PL_OK:
+        raise PLError(status, what)
+
+
+# --------------------------------------------------------------------------- helpers
+
+def _ptr(t) -> int | None:
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream) or None
+    return int(getattr(stream, "cuda_stream", stream)) or None
+
+
+def _ptr_array(ts):
+    arr = (vp * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = _ptr(t)
+    return arr
+
+
+def _contig(t, name):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+# --------------------------------------------------------------------------- primitives
+
+def gemm(a, b, out=None, stream=None):
+    """out[M,N] = a[M,K] @ b[K,N] (fp16, fp32 accumulate) on tcgen05."""
+    import torch
+    M, K = a.shape
+    N = b.shape[1]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=a.device)
+    check(lib.pl_gemm_f16(_ptr(a), a.stride(0), _ptr(b), b.stride(0), _ptr(out), out.stride(0),
+                          M, N, K, _stream(stream)), "pl_gemm_f16")
+    return out
+
+
+def segment_attention(q, segments, heads, head_dim, out=None, stream=None):
+    """Attention of q [F, Nq, ld] over KV segments (k, v, frame_shared) without concatenation.
+
+    Each segment is (k, v) with k/v [F, L, ld] (per-frame) or [L, ld] (shared).
+    """
+    import torch
+    F, Nq = q.shape[0], q.shape[1]
+    segs = (KVSegment * len(segments))()
+    for i, (k, v) in enumerate(segments):
+        if k.dim() == 3:
+            segs[i] = KVSegment(_ptr(k), _ptr(v), k.shape[1], k.stride(1), k.stride(0))
+        else:
+            segs[i] = KVSegment(_ptr(k), _ptr(v), k.shape[0], k.stride(0), 0)
+    if out is None:
+        out = torch.empty((F, Nq, heads * head_dim), dtype=torch.float16, device=q.device)
+    check(lib.pl_segment_attention(_ptr(q), q.stride(1), q.stride(0), segs, len(segments), F, Nq,
+                                   heads, head_dim, _ptr(out), out.stride(1), out.stride(0),
+                                   _stream(stream)), "pl_segment_attention")
+    return out
+
+
+def ref_attention(hidden, w_qkv, w_o, bank_feats, heads, out=None, workspace=None, stream=None):
+    """Reference attention layer: hidden [F,N,C], bank_feats list of [N,C]."""
+    import torch
+    F, N, Cc = hidden.shape
+    nb = len(bank_feats)
+    need = sz()
+    check(lib.pl_ref_attention_workspace_bytes(F, N, Cc, nb, C.byref(need)), "workspace")
+    if workspace is None:
+        workspace = torch.empty(need.value, dtype=torch.uint8, device=hidden.device)
+    if out is None:
+        out = torch.empty_like(hidden)
+    arr = _ptr_array(bank_feats) if nb else None
+    check(lib.pl_ref_attention(_ptr(_contig(hidden, "hidden")), _ptr(w_qkv), _ptr(w_o), arr, nb, F,
+                               N, Cc, heads, _ptr(out), _ptr(workspace), workspace.numel(),
+                               _stream(stream)), "pl_ref_attention")
+    return out
+
+
+def motion_xattn(x, motion, m_q, m_kv, m_o, heads, out=None, workspace=None, stream=None):
+    """Motion cross-attention: x [F,N,C] fp16, motion [F,512] fp32."""
+    import torch
+    F, N, Cc = x.shape
+    need = sz()
+    check(lib.pl_motion_xattn_workspace_bytes(F, N, Cc, C.byref(need)), "workspace")
+    if workspace is None:
+        workspace = torch.empty(need.value, dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty_like(x)
+    check(lib.pl_motion_xattn(_ptr(_contig(x, "x")), _ptr(motion), _ptr(m_q), _ptr(m_kv),
+                              _ptr(m_o), F, N, Cc, heads, _ptr(out), _ptr(workspace),
+                              workspace.numel(), _stream(stream)), "pl_motion_xattn")
+    return out
+
+
+def motion_bank_check(bank, count, appends, queries, threshold, cap, argmin=None, min_d2=None,
+                      appended=None, stream=None):
+    """In-order bank check; bank [capacity, dim] fp32, count/appends int32 [1] (device state)."""
+    cap_, dim = bank.shape
+    nq = queries.shape[0]
+    check(lib.pl_motion_bank_check(_ptr(bank), _ptr(count), _ptr(appends), cap_, dim,
+                                   _ptr(queries), nq, float(threshold), int(cap), _ptr(argmin),
+                                   _ptr(min_d2), _ptr(appended), _stream(stream)),
+          "pl_motion_bank_check")
+
+
+# --------------------------------------------------------------------------- stream context
+
+def make_config(latent_hw=(64, 64), layers=(), heads=8, threshold=17.0, append_cap=3, latent_c=4):
+    """layers: sequence of (tokens N, channels C)."""
+    cfg = Config()
+    cfg.latent_c, (cfg.latent_h, cfg.latent_w) = latent_c, latent_hw
+    cfg.n_layers = len(layers)
+    for i, (n, c) in enumerate(layers):
+        cfg.layer_tokens[i] = n
+        cfg.layer_channels[i] = c
+    cfg.heads = heads
+    cfg.drift_threshold = threshold
+    cfg.append_cap = append_cap
+    return cfg
+
+
+class Stream:
+    """One PersonaLive stream: the device-resident pile and the reference bank."""
+
+    def __init__(self, cfg: Config, device="cuda"):
+        import torch
+        self.cfg = cfg
+        need = sz()
+        check(lib.pl_workspace_bytes(C.byref(cfg), C.byref(need)), "pl_workspace_bytes")
+        self.workspace = torch.empty(need.value, dtype=torch.uint8, device=device)
+        h = vp()
+        check(lib.pl_ctx_create(C.byref(cfg), _ptr(self.workspace), need.value, C.byref(h)),
+              "pl_ctx_create")
+        self.handle = h
+        self._keep = []
+
+    def close(self):
+        if self.handle:
+            lib.pl_ctx_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def bank_init(self, weights, ref_feats, anchor_feats, ref_motion, drive0_motion, ref_latent,
+                  prefill_eps, stream=None):
+        """weights: list of dicts with w_qkv, w_o, m_q, m_kv, m_o (device fp16)."""
+        L = self.cfg.n_layers
+        wa = (LayerWeights * max(L, 1))()
+        for i, w in enumerate(weights[:L]):
+            wa[i] = LayerWeights(_ptr(w["w_qkv"]), _ptr(w["w_o"]), _ptr(w["m_q"]),
+                                 _ptr(w["m_kv"]), _ptr(w["m_o"]))
+        rf = _ptr_array(ref_feats) if L else None
+        af = _ptr_array(anchor_feats) if anchor_feats else None
+        self._keep = [weights, ref_feats, anchor_feats, ref_motion, drive0_motion, ref_latent,
+                      prefill_eps]
+        check(lib.pl_bank_init(self.handle, wa if L else None, rf, af, _ptr(ref_motion),
+                               _ptr(drive0_motion), _ptr(ref_latent), _ptr(prefill_eps),
+                               _stream(stream)), "pl_bank_init")
+
+    def ring_push(self, new_noise, new_motion, stream=None):
+        check(lib.pl_ring_push(self.handle, _ptr(new_noise), _ptr(new_motion), _stream(stream)),
+              "pl_ring_push")
+
+    def ddim_step(self, eps, out_x0, stream=None):
+        check(lib.pl_pyramid_ddim_step(self.handle, _ptr(eps), _ptr(out_x0), _stream(stream)),
+              "pl_pyramid_ddim_step")
+
+    def bank_check(self, queries, argmin=None, min_d2=None, appended=None, stream=None):
+        check(lib.pl_ctx_bank_check(self.handle, _ptr(queries), queries.shape[0], _ptr(argmin),
+                                    _ptr(min_d2), _ptr(appended), _stream(stream)),
+              "pl_ctx_bank_check")
+
+    def round(self, new_noise, new_motion, hidden, eps, out_frames, appended=None,
+              layer_out=None, stream=None):
+        L = self.cfg.n_layers
+        hp = _ptr_array(hidden) if L else None
+        lo = _ptr_array(layer_out) if layer_out is not None else None
+        check(lib.pl_stream_round(self.handle, _ptr(new_noise), _ptr(new_motion), hp, _ptr(eps),
+                                  _ptr(out_frames), _ptr(appended), lo, _stream(stream)),
+              "pl_stream_round")
+
+    def state(self, stream=None):
+        s = State()
+        check(lib.pl_get_state(self.handle, C.byref(s), _stream(stream)), "pl_get_state")
+        return s.as_dict()
+
+    def motion_bank(self, stream=None):
+        import numpy as np
+        buf = np.zeros((4, 512), dtype=np.float32)
+        n = C.c_int32()
+        check(lib.pl_get_motion_bank(self.handle, buf.ctypes.data, C.byref(n), _stream(stream)),
+              "pl_get_motion_bank")
+        return buf[: n.value].copy()
+
+    def device_status(self, stream=None) -> int:
+        return lib.pl_get_device_status(self.handle, _stream(stream))
+
+    def ring_latents(self):
+        return lib.pl_ctx_ring_latents(self.handle)

@@ -1,0 +1,43 @@
+// Flash-style attention over a list of KV segments on tcgen05 tensor cores.
+#pragma once
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace pl {
+
+constexpr int kAttnMaxSegs = 8;
+
+struct AttnSeg {
+  CUtensorMap k;   // 4D {head_dim, heads, len, frames|1}, box {64, 1, BN, 1}
+  CUtensorMap v;
+  int len;
+  int per_frame;   // 1: frame f reads its own rows, 0: shared by all frames
+};
+
+struct AttnParams {
+  CUtensorMap q;               // 4D {head_dim, heads, n_q, frames}, box {64, 1, 128, 1}
+  AttnSeg seg[kAttnMaxSegs];
+  int n_fixed;                 // segments always attended
+  int n_total;                 // segments available
+  const int32_t* n_extra;      // when non-null: attend n_fixed + min(*n_extra, n_total - n_fixed)
+  __half* out;
+  int64_t ldo, out_fstride;
+  int n_q, heads, frames;
+  float scale_log2;            // log2(e) / sqrt(head_dim)
+  uint32_t* status;
+};
+
+struct AttnSegHost {
+  const void* k;
+  const void* v;
+  int64_t len, ld, frame_stride;
+};
+
+// Build params (tensor maps) on the host. Returns 0 on success.
+int attn_make_params(AttnParams* p, const void* q, int64_t ldq, int64_t q_fstride,
+                     const AttnSegHost* segs, int n_segs, int frames, int n_q, int heads,
+                     int head_dim, void* out, int64_t ldo, int64_t out_fstride);
+int attn_launch(const AttnParams& p, int head_dim, cudaStream_t stream);
+
+}  // namespace pl

@@ -1,0 +1,251 @@
+// Persistent, warp-specialised fp16 GEMM on tcgen05 tensor cores.
+//
+//   warp 0      TMA producer: A tile [128 x 64] (K-major) + B tile [64 x BN]
+//               (MN-major, BN/64 column blocks), 128-byte swizzle, STAGES ring
+//   warp 1      MMA issuer (one lane): 4 x tcgen05.mma (K = 16) per stage into
+//               a TMEM accumulator; two accumulators alternate between tiles
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
+//               row), fp32 -> fp16, 16-byte stores
+#include <cuda_runtime.h>
+
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "tmap.cuh"
+
+namespace pl {
+
+namespace {
+
+constexpr int kStages = 5;
+constexpr int kNB = (kGemmBN + 63) / 64;            // 64-column B blocks per tile
+constexpr uint32_t kABytes = kGemmBM * 128;          // 128 rows x 128 B
+constexpr uint32_t kBBlockBytes = 64 * 128;          // 64 K-rows x 128 B
+constexpr uint32_t kBBytes = kNB * kBBlockBytes;
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kAccStride = 256;                 // TMEM columns per accumulator
+constexpr int kThreads = 192;
+constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
+
+struct TileCoord {
+  int prob, m0, n0;
+};
+
+__device__ __forceinline__ bool decode_tile(const GemmParams& p, int t, TileCoord& tc) {
+  int pi = 0;
+  while (pi < p.n_problems - 1 && t >= p.prob[pi].tile_end) ++pi;
+  const GemmProblem& pr = p.prob[pi];
+  if (pr.pred != nullptr && *((volatile const int32_t*)pr.pred) == 0) return false;
+  const int local = t - pr.tile_begin;
+  tc.prob = pi;
+  tc.m0 = (local / pr.tiles_n) * kGemmBM;
+  tc.n0 = (local % pr.tiles_n) * kGemmBN;
+  return true;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < p.n_problems; ++i) {
+        tma_prefetch_desc(&p.prob[i].a);
+        tma_prefetch_desc(&p.prob[i].b);
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = blockIdx.x; t < p.total_tiles && !*abort_flag; t += gridDim.x) {
+        TileCoord tc;
+        if (!decode_tile(p, t, tc)) continue;
+        const GemmProblem& pr = p.prob[tc.prob];
+        const int nk = (pr.K + kGemmBK - 1) / kGemmBK;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+          uint8_t* sa = smem + stage * kStageBytes;
+          uint8_t* sb = sa + kABytes;
+          mbar_expect_tx(&full[stage], kStageBytes);
+          tma_load_2d(sa, &pr.a, &full[stage], kb * kGemmBK, tc.m0);
+#pragma unroll
+          for (int j = 0; j < kNB; ++j)
+            tma_load_2d(sb + j * kBBlockBytes, &pr.b, &full[stage], tc.n0 + 64 * j, kb * kGemmBK);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(kGemmBM, kGemmBN, 0, 1);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc_i = 0;
+      for (int t = blockIdx.x; t < p.total_tiles && !*abort_flag; t += gridDim.x) {
+        TileCoord tc;
+        if (!decode_tile(p, t, tc)) continue;
+        const GemmProblem& pr = p.prob[tc.prob];
+        const int nk = (pr.K + kGemmBK - 1) / kGemmBK;
+        const int buf = acc_i & 1;
+        const uint32_t use = static_cast<uint32_t>(acc_i >> 1);
+        if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * kAccStride;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * kStageBytes);
+          const uint32_t b0 = a0 + kABytes;
+#pragma unroll
+          for (int k = 0; k < kGemmBK / 16; ++k) {
+            const uint64_t ad = desc_sw128(a0 + 32 * k, 16, 1024);
+            const uint64_t bd = desc_sw128(b0 + 2048 * k, kBBlockBytes, 1024);
+            mma_ss(d, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        mma_commit(&acc_full[buf]);
+        ++acc_i;
+      }
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;   // TMEM lane quadrant this warp may access
+    const int row_in_tile = 32 * q + lane;
+    int acc_i = 0;
+    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+      TileCoord tc;
+      if (!decode_tile(p, t, tc)) continue;
+      const GemmProblem& pr = p.prob[tc.prob];
+      const int buf = acc_i & 1;
+      const uint32_t use = static_cast<uint32_t>(acc_i >> 1);
+      if (!mbar_wait(&acc_full[buf], use & 1, abort_flag)) break;
+      tc_fence_after();
+      const int row = tc.m0 + row_in_tile;
+      const uint32_t taddr = tmem + buf * kAccStride + (static_cast<uint32_t>(32 * q) << 16);
+      __half* crow = pr.c + static_cast<int64_t>(row) * pr.ldc;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr + c0, r);
+        tmem_wait_ld();
+        const int col = tc.n0 + c0;
+        if (row < pr.M && col < pr.N) {
+          uint4 v0, v1;
+          v0.x = pack_half2(__uint_as_float(r[0]), __uint_as_float(r[1]));
+          v0.y = pack_half2(__uint_as_float(r[2]), __uint_as_float(r[3]));
+          v0.z = pack_half2(__uint_as_float(r[4]), __uint_as_float(r[5]));
+          v0.w = pack_half2(__uint_as_float(r[6]), __uint_as_float(r[7]));
+          v1.x = pack_half2(__uint_as_float(r[8]), __uint_as_float(r[9]));
+          v1.y = pack_half2(__uint_as_float(r[10]), __uint_as_float(r[11]));
+          v1.z = pack_half2(__uint_as_float(r[12]), __uint_as_float(r[13]));
+          v1.w = pack_half2(__uint_as_float(r[14]), __uint_as_float(r[15]));
+          uint4* dst = reinterpret_cast<uint4*>(crow + col);
+          dst[0] = v0;
+          dst[1] = v1;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+      ++acc_i;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && *abort_flag && p.status) atomicOr(p.status, DEV_TIMEOUT);
+}
+
+}  // namespace
+
+int gemm_make_problem(GemmProblem* p, const void* a, int64_t lda, const void* b, int64_t ldb,
+                      void* c, int64_t ldc, int M, int N, int K, const int32_t* pred) {
+  if (M <= 0 || N <= 0 || K <= 0) return 1;
+  if (N % 16 || K % 8 || lda % 8 || ldb % 8 || ldc % 8) return 1;
+  if (lda < K || ldb < N || ldc < N) return 1;
+  if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b) |
+       reinterpret_cast<uintptr_t>(c)) & 15)
+    return 1;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(lda) * 2};
+    const uint32_t box[2] = {64, kGemmBM};
+    if (encode_f16_tmap(&p->a, a, 2, dims, strides, box) != 0) return 2;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(ldb) * 2};
+    const uint32_t box[2] = {64, 64};
+    if (encode_f16_tmap(&p->b, b, 2, dims, strides, box) != 0) return 2;
+  }
+  p->c = static_cast<__half*>(c);
+  p->ldc = ldc;
+  p->M = M;
+  p->N = N;
+  p->K = K;
+  p->tiles_n = (N + kGemmBN - 1) / kGemmBN;
+  p->pred = pred;
+  return 0;
+}
+
+int gemm_launch(GemmParams* params, cudaStream_t stream, int max_ctas) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(gemm_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+      return 4;
+    attr_done = true;
+  }
+  int total = 0;
+  for (int i = 0; i < params->n_problems; ++i) {
+    GemmProblem& pr = params->prob[i];
+    const int tiles_m = (pr.M + kGemmBM - 1) / kGemmBM;
+    pr.tile_begin = total;
+    total += tiles_m * pr.tiles_n;
+    pr.tile_end = total;
+  }
+  params->total_tiles = total;
+  if (total == 0) return 0;
+  int grid = total < max_ctas ? total : max_ctas;
+  gemm_f16_kernel<<<grid, kThreads, kSmemBytes, stream>>>(*params);
+  return cudaGetLastError() == cudaSuccess ? 0 : 4;
+}
+
+}  // namespace pl

@@ -1,0 +1,439 @@
+#include <cmath>
+
+#include "misc.cuh"
+#include "ptx.cuh"
+
+namespace pl {
+
+// ------------------------------------------------------------------ schedule
+// SD scaled-linear betas (beta_i = (sqrt(0.00085) + i (sqrt(0.012) -
+// sqrt(0.00085)) / 999)^2), alpha_bar_t = prod_{i<=t} (1 - beta_i), in fp64.
+void ddim_coefficients(DdimCoef* out) {
+  double abar[1000];
+  const double a = std::sqrt(0.00085), b = std::sqrt(0.012);
+  double prod = 1.0;
+  for (int i = 0; i < 1000; ++i) {
+    const double r = a + i * (b - a) / 999.0;
+    prod *= 1.0 - r * r;
+    abar[i] = prod;
+  }
+  const int ts[4] = {999, 666, 333, 0};
+  for (int k = 0; k < 4; ++k) {
+    const int t = ts[k];
+    const double at = abar[t];
+    const double ap = t - 333 >= 0 ? abar[t - 333] : 1.0;
+    out->c[k][0] = std::sqrt(at);
+    out->c[k][1] = std::sqrt(1.0 - at);
+    out->c[k][2] = std::sqrt(ap);
+    out->c[k][3] = std::sqrt(1.0 - ap);
+  }
+}
+
+namespace {
+
+__device__ __forceinline__ int t_index(int t) {  // 999 -> 0, 666 -> 1, 333 -> 2, 0 -> 3
+  return t == 999 ? 0 : t == 666 ? 1 : t == 333 ? 2 : t == 0 ? 3 : -1;
+}
+
+// ------------------------------------------------------------------ prefill
+// 3 windows at t = 0, 333, 666 (oldest first) in slots 0..2; slot 3 free.
+__global__ void prefill_kernel(DevState* st, float* ring, float* slot_motion, float* bank,
+                               const float* __restrict__ ref_latent,
+                               const float* __restrict__ prefill_eps,
+                               const float* __restrict__ ref_motion,
+                               const float* __restrict__ drive0, int64_t frame_elems,
+                               DdimCoef coef) {
+  const int64_t total = 12 * frame_elems;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t k = i / frame_elems;      // prefill frame 0..11
+    const int64_t e = i - k * frame_elems;
+    const int w = static_cast<int>(k / 4);  // window 0..2 -> t = 0, 333, 666
+    const int ti = 3 - w;                   // table index of t
+    const double x = coef.c[ti][0] * static_cast<double>(ref_latent[e]) +
+                     coef.c[ti][1] * static_cast<double>(prefill_eps[i]);
+    ring[i] = static_cast<float>(x);        // slot w, frame k % 4
+  }
+  // motion: 13-point ramp ref -> drive0 with the last point dropped
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < 12 * 512;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int k = static_cast<int>(i / 512);
+    const int d = static_cast<int>(i % 512);
+    const double r = ref_motion[d], t = drive0[d];
+    slot_motion[i] = static_cast<float>(r + (static_cast<double>(k) / 12.0) * (t - r));
+  }
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < 512;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    bank[i] = ref_motion[i];
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    st->head = 0;
+    st->slot_t[0] = 0;
+    st->slot_t[1] = 333;
+    st->slot_t[2] = 666;
+    st->slot_t[3] = -1;
+    st->bank_count = 1;
+    st->appends = 0;
+    st->kv_extra = 0;
+    for (int a = 0; a < 4; ++a) st->anchor_fire[a] = 0;
+    st->rounds = 0;
+    st->frames_in = 0;
+    st->frames_out = 0;
+    st->initialised = 1;
+  }
+}
+
+// ------------------------------------------------------------------ ring push
+__global__ void ring_push_kernel(DevState* st, float* ring, float* slot_motion,
+                                 float* batch_motion, const float* __restrict__ new_noise,
+                                 const float* __restrict__ new_motion, int64_t frame_elems) {
+  const int head = st->head;
+  const int slot = (head + 3) & 3;
+  const int64_t n4 = 4 * frame_elems / 4;
+  float4* dst = reinterpret_cast<float4*>(ring + slot * 4 * frame_elems);
+  const float4* src = reinterpret_cast<const float4*>(new_noise);
+  const int64_t tid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int64_t nthr = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = tid; i < n4; i += nthr) dst[i] = src[i];
+  // per-slot motion of the new window, and the batch's motion in batch order
+  for (int64_t i = tid; i < 16 * 512; i += nthr) {
+    const int f = static_cast<int>(i / 512);
+    const int w = f >> 2;
+    const int s = (head + w) & 3;
+    const int64_t off = (static_cast<int64_t>(s) * 4 + (f & 3)) * 512 + (i % 512);
+    float v;
+    if (w == 3) {
+      v = new_motion[(f & 3) * 512 + (i % 512)];
+      slot_motion[off] = v;
+    } else {
+      v = slot_motion[off];
+    }
+    batch_motion[i] = v;
+  }
+  if (tid == 0) {
+    if (st->slot_t[slot] != -1) atomicOr(&st->status, DEV_BADARG);
+    st->slot_t[slot] = 999;
+    st->frames_in += 4;
+  }
+}
+
+// ------------------------------------------------------------------ DDIM
+// Batch frame f belongs to window w = f / 4 (oldest first), physical slot
+// (head + w) & 3. Arithmetic in fp64, one rounding to fp32 per output.
+__global__ void ddim_kernel(const DevState* __restrict__ st, float* ring,
+                            const float* __restrict__ eps, float* __restrict__ out_x0,
+                            int64_t frame_elems, DdimCoef coef) {
+  const int head = st->head;
+  int tix[4], slot[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    slot[w] = (head + w) & 3;
+    tix[w] = t_index(st->slot_t[slot[w]]);
+  }
+  const int64_t fe4 = frame_elems / 4;
+  const int64_t total = 16 * fe4;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int f = static_cast<int>(i / fe4);
+    const int64_t e = i - f * fe4;
+    const int w = f >> 2, j = f & 3;
+    const int ti = tix[w];
+    if (ti < 0) continue;
+    float4* xp = reinterpret_cast<float4*>(ring) + (static_cast<int64_t>(slot[w]) * 4 + j) * fe4 + e;
+    const float4 x = *xp;
+    const float4 ep = reinterpret_cast<const float4*>(eps)[i];
+    const double sa = coef.c[ti][0], sb = coef.c[ti][1];
+    const double x0x = (x.x - sb * ep.x) / sa, x0y = (x.y - sb * ep.y) / sa;
+    const double x0z = (x.z - sb * ep.z) / sa, x0w = (x.w - sb * ep.w) / sa;
+    if (ti == 3) {
+      reinterpret_cast<float4*>(out_x0)[j * fe4 + e] =
+          make_float4(static_cast<float>(x0x), static_cast<float>(x0y), static_cast<float>(x0z),
+                      static_cast<float>(x0w));
+    } else {
+      const double pa = coef.c[ti][2], pb = coef.c[ti][3];
+      *xp = make_float4(static_cast<float>(pa * x0x + pb * ep.x),
+                        static_cast<float>(pa * x0y + pb * ep.y),
+                        static_cast<float>(pa * x0z + pb * ep.z),
+                        static_cast<float>(pa * x0w + pb * ep.w));
+    }
+  }
+}
+
+__global__ void ring_commit_kernel(DevState* st) {
+  int popped = 0;
+  for (int s = 0; s < 4; ++s) {
+    const int t = st->slot_t[s];
+    if (t == 0) {
+      st->slot_t[s] = -1;
+      ++popped;
+    } else if (t > 0) {
+      st->slot_t[s] = t - 333;
+    }
+  }
+  if (popped != 1) atomicOr(&st->status, DEV_BADARG);
+  st->head = (st->head + 1) & 3;
+  st->rounds += 1;
+  st->frames_out += 4;
+}
+
+// ------------------------------------------------------------------ bank check
+constexpr int kBankThreads = 256;
+
+__global__ void __launch_bounds__(kBankThreads) bank_check_kernel(
+    float* bank, int32_t* count_p, int32_t* appends_p, int capacity, int dim,
+    const float* __restrict__ queries, int nq, double thr2, int cap, int32_t* argmin,
+    double* min_d2, uint8_t* appended, DevState* st) {
+  __shared__ double w_best[kBankThreads / 32];
+  __shared__ int w_idx[kBankThreads / 32];
+  __shared__ int s_cnt, s_app, s_do_append;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int nwarps = kBankThreads / 32;
+  if (threadIdx.x == 0) {
+    s_cnt = *count_p;
+    s_app = *appends_p;
+    if (st) {
+      for (int a = 0; a < 4; ++a) st->anchor_fire[a] = 0;
+    }
+  }
+  __syncthreads();
+  for (int qi = 0; qi < nq; ++qi) {
+    const float* q = queries + static_cast<int64_t>(qi) * dim;
+    const int cnt = s_cnt;
+    double best = INFINITY;
+    int bidx = 0x7fffffff;
+    for (int j = warp; j < cnt; j += nwarps) {
+      const float* b = bank + static_cast<int64_t>(j) * dim;
+      double acc = 0.0;
+      for (int d = lane; d < dim; d += 32) {
+        const double diff = static_cast<double>(q[d]) - static_cast<double>(b[d]);
+        acc = fma(diff, diff, acc);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (acc < best) {  // j increases, so the first minimum is kept
+        best = acc;
+        bidx = j;
+      }
+    }
+    if (lane == 0) {
+      w_best[warp] = best;
+      w_idx[warp] = bidx;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double b = INFINITY;
+      int bi = 0x7fffffff;
+      for (int w = 0; w < nwarps; ++w) {
+        if (w_best[w] < b || (w_best[w] == b && w_idx[w] < bi)) {
+          b = w_best[w];
+          bi = w_idx[w];
+        }
+      }
+      if (bi == 0x7fffffff) bi = -1;
+      if (argmin) argmin[qi] = bi;
+      if (min_d2) min_d2[qi] = b;
+      const int doit = (cnt > 0 && b > thr2 && s_app < cap && cnt < capacity) ? 1 : 0;
+      s_do_append = doit;
+      if (appended) appended[qi] = static_cast<uint8_t>(doit);
+    }
+    __syncthreads();
+    if (s_do_append) {
+      float* dst = bank + static_cast<int64_t>(cnt) * dim;
+      for (int d = threadIdx.x; d < dim; d += kBankThreads) dst[d] = q[d];
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        s_cnt = cnt + 1;
+        s_app = s_app + 1;
+        if (st && s_app < 4) st->anchor_fire[s_app] = 1;
+      }
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    *count_p = s_cnt;
+    *appends_p = s_app;
+  }
+}
+
+// ------------------------------------------------------------------ motion
+struct PeTable {
+  float v[32][16];
+};
+
+// tokens[f][p][c] = fp16(motion[f][16 p + c] + PE[p][c]);
+// kv[f][p][n] = sum_c tokens[f][p][c] * m_kv[c][n] (fp32 accumulate), n < 2C.
+__global__ void motion_kv_kernel(const float* __restrict__ motion, const __half* __restrict__ m_kv,
+                                 int C, __half* tokens, __half* kv, PeTable pe) {
+  __shared__ float tok[32][16];
+  const int f = blockIdx.y;
+  for (int i = threadIdx.x; i < 512; i += blockDim.x) {
+    const int p = i >> 4, c = i & 15;
+    const __half h = __float2half_rn(motion[f * 512 + i] + pe.v[p][c]);
+    tok[p][c] = __half2float(h);
+    if (blockIdx.x == 0) tokens[f * 512 + i] = h;
+  }
+  __syncthreads();
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= 2 * C) return;
+  float w[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) w[c] = __half2float(m_kv[c * 2 * C + n]);
+  for (int p = 0; p < 32; ++p) {
+    float acc = 0.f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) acc = fmaf(tok[p][c], w[c], acc);
+    kv[(static_cast<int64_t>(f) * 32 + p) * 2 * C + n] = __float2half_rn(acc);
+  }
+}
+
+// One thread per (query row, head): 32 scores in registers, smem-resident
+// K/V of the frame and head (fp32), softmax in fp32.
+template <int HD>
+__global__ void __launch_bounds__(128) motion_attn_kernel(const __half* __restrict__ q, int64_t ldq,
+                                                          const __half* __restrict__ kv, int N,
+                                                          int C, __half* __restrict__ out,
+                                                          int64_t ldo, float scale) {
+  __shared__ float sk[32][HD];
+  __shared__ float sv[32][HD];
+  const int f = blockIdx.z, h = blockIdx.y;
+  const __half* kvf = kv + static_cast<int64_t>(f) * 32 * 2 * C;
+  for (int i = threadIdx.x; i < 32 * HD; i += blockDim.x) {
+    const int p = i / HD, d = i % HD;
+    sk[p][d] = __half2float(kvf[p * 2 * C + h * HD + d]);
+    sv[p][d] = __half2float(kvf[p * 2 * C + C + h * HD + d]);
+  }
+  __syncthreads();
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  const __half* qr = q + (static_cast<int64_t>(f) * N + n) * ldq + h * HD;
+  float s[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) s[j] = 0.f;
+  for (int d0 = 0; d0 < HD; d0 += 8) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(qr + d0);
+    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+    float qv[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 t = __half22float2(h2[e]);
+      qv[2 * e] = t.x;
+      qv[2 * e + 1] = t.y;
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s[j] = fmaf(qv[e], sk[j][d0 + e], s[j]);
+    }
+  }
+  float mx = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    s[j] *= scale;
+    mx = fmaxf(mx, s[j]);
+  }
+  float sum = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    s[j] = __expf(s[j] - mx);
+    sum += s[j];
+  }
+  const float inv = 1.f / sum;
+  __half* orow = out + (static_cast<int64_t>(f) * N + n) * ldo + h * HD;
+  for (int d0 = 0; d0 < HD; d0 += 8) {
+    float o[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = fmaf(s[j], sv[j][d0 + e], o[e]);
+    }
+    uint4 r;
+    r.x = pack_half2(o[0] * inv, o[1] * inv);
+    r.y = pack_half2(o[2] * inv, o[3] * inv);
+    r.z = pack_half2(o[4] * inv, o[5] * inv);
+    r.w = pack_half2(o[6] * inv, o[7] * inv);
+    *reinterpret_cast<uint4*>(orow + d0) = r;
+  }
+}
+
+int grid_for(int64_t work, int threads) {
+  int64_t g = (work + threads - 1) / threads;
+  const int64_t cap = 148 * 16;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(DevState* st, float* ring, float* slot_motion, float* bank,
+                           const float* ref_latent, const float* prefill_eps,
+                           const float* ref_motion, const float* drive0, int64_t frame_elems,
+                           cudaStream_t s) {
+  DdimCoef coef;
+  ddim_coefficients(&coef);
+  prefill_kernel<<<grid_for(12 * frame_elems, 256), 256, 0, s>>>(
+      st, ring, slot_motion, bank, ref_latent, prefill_eps, ref_motion, drive0, frame_elems, coef);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ring_push(DevState* st, float* ring, float* slot_motion, float* batch_motion,
+                             const float* new_noise, const float* new_motion,
+                             int64_t frame_elems, cudaStream_t s) {
+  ring_push_kernel<<<grid_for(frame_elems, 256), 256, 0, s>>>(st, ring, slot_motion, batch_motion,
+                                                             new_noise, new_motion, frame_elems);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ddim(DevState* st, float* ring, const float* eps, float* out_x0,
+                        int64_t frame_elems, const DdimCoef& coef, cudaStream_t s) {
+  ddim_kernel<<<grid_for(4 * frame_elems, 256), 256, 0, s>>>(st, ring, eps, out_x0, frame_elems,
+                                                            coef);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ring_commit(DevState* st, cudaStream_t s) {
+  ring_commit_kernel<<<1, 1, 0, s>>>(st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bank_check(float* bank, int32_t* count, int32_t* appends, int capacity,
+                              int dim, const float* queries, int nq, double thr2, int cap,
+                              int32_t* argmin, double* min_d2, uint8_t* appended,
+                              DevState* st, cudaStream_t s) {
+  bank_check_kernel<<<1, kBankThreads, 0, s>>>(bank, count, appends, capacity, dim, queries, nq,
+                                               thr2, cap, argmin, min_d2, appended, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_motion_kv(const float* motion, const __half* m_kv, int F, int C,
+                             __half* tokens, __half* kv, cudaStream_t s) {
+  PeTable pe;
+  for (int p = 0; p < 32; ++p)
+    for (int i = 0; i < 8; ++i) {
+      const double ang = p / std::pow(10000.0, 2.0 * i / 16.0);
+      pe.v[p][2 * i] = static_cast<float>(std::sin(ang));
+      pe.v[p][2 * i + 1] = static_cast<float>(std::cos(ang));
+    }
+  dim3 grid((2 * C + 255) / 256, F);
+  motion_kv_kernel<<<grid, 256, 0, s>>>(motion, m_kv, C, tokens, kv, pe);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_motion_attn(const __half* q, int64_t ldq, const __half* kv, int F, int N,
+                               int C, int heads, __half* out, int64_t ldo, cudaStream_t s) {
+  const int hd = C / heads;
+  dim3 grid((N + 127) / 128, heads, F);
+  const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(hd)));
+  switch (hd) {
+    case 40: motion_attn_kernel<40><<<grid, 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
+    case 64: motion_attn_kernel<64><<<grid, 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
+    case 80: motion_attn_kernel<80><<<grid, 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
+    case 128: motion_attn_kernel<128><<<grid, 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
+    case 160: motion_attn_kernel<160><<<grid, 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace pl

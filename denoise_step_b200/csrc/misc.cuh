@@ -1,0 +1,57 @@
+// Streaming kernels of the round: pile (ring) maintenance, the pyramid DDIM
+// step, the motion-bank check and the motion cross-attention pieces.
+#pragma once
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace pl {
+
+// Device-resident state of one stream (lives in the context's workspace).
+struct DevState {
+  int32_t head;            // physical slot of the oldest window
+  int32_t slot_t[4];       // timestep per slot, -1 = free
+  int32_t bank_count;      // motion-bank entries
+  int32_t appends;         // anchors appended so far
+  int32_t kv_extra;        // KV-bank entries beyond the reference (anchors projected)
+  int32_t anchor_fire[4];  // [a] = 1 when anchor a was appended by the latest bank check
+  int32_t initialised;
+  int32_t pad_;
+  int64_t rounds, frames_in, frames_out;
+  uint32_t status;
+  uint32_t pad2_[3];
+};
+
+// Per-timestep DDIM coefficients for the 4 timesteps of the table, in table
+// order t = 999, 666, 333, 0: {sqrt(abar_t), sqrt(1-abar_t), sqrt(abar_prev),
+// sqrt(1-abar_prev)} with abar_prev = 1 below t = 0.
+struct DdimCoef {
+  double c[4][4];
+};
+
+// Host: fill the coefficients from the SD scaled-linear schedule.
+void ddim_coefficients(DdimCoef* out);
+
+// Host launchers. frame_elems = latent_c * H * W (multiple of 4).
+cudaError_t launch_prefill(DevState* st, float* ring, float* slot_motion, float* bank,
+                           const float* ref_latent, const float* prefill_eps,
+                           const float* ref_motion, const float* drive0, int64_t frame_elems,
+                           cudaStream_t s);
+cudaError_t launch_ring_push(DevState* st, float* ring, float* slot_motion, float* batch_motion,
+                             const float* new_noise, const float* new_motion,
+                             int64_t frame_elems, cudaStream_t s);
+cudaError_t launch_ddim(DevState* st, float* ring, const float* eps, float* out_x0,
+                        int64_t frame_elems, const DdimCoef& coef, cudaStream_t s);
+cudaError_t launch_ring_commit(DevState* st, cudaStream_t s);
+cudaError_t launch_bank_check(float* bank, int32_t* count, int32_t* appends, int capacity,
+                              int dim, const float* queries, int nq, double thr2, int cap,
+                              int32_t* argmin, double* min_d2, uint8_t* appended,
+                              DevState* st, cudaStream_t s);
+// tokens (fp16 [F][32][16]) and motion K/V (fp16 [F][32][2C]) of every frame.
+cudaError_t launch_motion_kv(const float* motion, const __half* m_kv, int F, int C,
+                             __half* tokens, __half* kv, cudaStream_t s);
+// out[f*N + n][h*hd + d] = softmax_j(q . k_j / sqrt(hd)) v_j, 32 keys per frame.
+cudaError_t launch_motion_attn(const __half* q, int64_t ldq, const __half* kv, int F, int N,
+                               int C, int heads, __half* out, int64_t ldo, cudaStream_t s);
+
+}  // namespace pl

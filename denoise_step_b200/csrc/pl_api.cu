@@ -1,0 +1,654 @@
+// C ABI (include/pl.h): argument validation, workspace layout, launch order
+// of one round and its CUDA-graph capture.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "../../include/pl.h"
+#include "attn.cuh"
+#include "gemm.cuh"
+#include "misc.cuh"
+#include "ptx.cuh"
+
+using pl::AttnParams;
+using pl::AttnSegHost;
+using pl::GemmParams;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
+}
+
+bool head_dim_supported(int hd) {
+  return hd == 40 || hd == 64 || hd == 80 || hd == 128 || hd == 160;
+}
+
+pl_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PL_OK : PL_ECUDA; }
+
+pl_status gemm_status(int r) {
+  return r == 0 ? PL_OK : r == 1 ? PL_EINVAL : r == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
+}
+
+}  // namespace
+
+// ====================================================================== context
+
+struct pl_ctx {
+  pl_config cfg;
+  int capacity;        // motion/KV bank capacity = 1 + append_cap
+  int64_t frame_elems; // latent_c * H * W
+  uint8_t* ws;
+  size_t ws_bytes;
+  pl::DevState* st;
+  float* ring;
+  float* slot_motion;
+  float* batch_motion;
+  float* bank;
+  __half* tokens;
+  __half* bank_kv[PL_MAX_LAYERS];
+  __half* motion_kv[PL_MAX_LAYERS];
+  __half* qkv;
+  __half* attn_o;
+  __half* a1;
+  __half* qm;
+  __half* om;
+  __half* out_default;
+  pl::DdimCoef coef;
+  bool initialised;
+  bool have_anchors;
+  pl_layer_weights w[PL_MAX_LAYERS];
+  const void* ref_feats[PL_MAX_LAYERS];
+  const void* anchor_feats[3][PL_MAX_LAYERS];
+  // captured round
+  cudaGraph_t graph;
+  cudaGraphExec_t exec;
+  const void* key[64];
+  int key_n;
+};
+
+namespace {
+
+// Workspace layout; with ctx == nullptr only the size is computed.
+size_t layout(const pl_config& c, pl_ctx* ctx) {
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> uint8_t* {
+    uint8_t* p = ctx ? ctx->ws + off : nullptr;
+    off += align_up(bytes);
+    return p;
+  };
+  const int capacity = 1 + c.append_cap;
+  const int64_t fe = static_cast<int64_t>(c.latent_c) * c.latent_h * c.latent_w;
+  uint8_t* st = take(sizeof(pl::DevState));
+  uint8_t* ring = take(sizeof(float) * 16 * fe);
+  uint8_t* sm = take(sizeof(float) * 16 * 512);
+  uint8_t* bm = take(sizeof(float) * 16 * 512);
+  uint8_t* bank = take(sizeof(float) * capacity * 512);
+  uint8_t* tok = take(sizeof(__half) * 16 * 32 * 16);
+  int64_t max_nc = 0;
+  for (int l = 0; l < c.n_layers; ++l) {
+    const int64_t N = c.layer_tokens[l], C = c.layer_channels[l];
+    uint8_t* bkv = take(sizeof(__half) * capacity * N * 2 * C);
+    uint8_t* mkv = take(sizeof(__half) * 16 * 32 * 2 * C);
+    if (ctx) {
+      ctx->bank_kv[l] = reinterpret_cast<__half*>(bkv);
+      ctx->motion_kv[l] = reinterpret_cast<__half*>(mkv);
+    }
+    if (16 * N * C > max_nc) max_nc = 16 * N * C;
+  }
+  uint8_t* qkv = take(sizeof(__half) * 3 * max_nc);
+  uint8_t* ao = take(sizeof(__half) * max_nc);
+  uint8_t* a1 = take(sizeof(__half) * max_nc);
+  uint8_t* qm = take(sizeof(__half) * max_nc);
+  uint8_t* om = take(sizeof(__half) * max_nc);
+  uint8_t* od = take(sizeof(__half) * max_nc);
+  if (ctx) {
+    ctx->st = reinterpret_cast<pl::DevState*>(st);
+    ctx->ring = reinterpret_cast<float*>(ring);
+    ctx->slot_motion = reinterpret_cast<float*>(sm);
+    ctx->batch_motion = reinterpret_cast<float*>(bm);
+    ctx->bank = reinterpret_cast<float*>(bank);
+    ctx->tokens = reinterpret_cast<__half*>(tok);
+    ctx->qkv = reinterpret_cast<__half*>(qkv);
+    ctx->attn_o = reinterpret_cast<__half*>(ao);
+    ctx->a1 = reinterpret_cast<__half*>(a1);
+    ctx->qm = reinterpret_cast<__half*>(qm);
+    ctx->om = reinterpret_cast<__half*>(om);
+    ctx->out_default = reinterpret_cast<__half*>(od);
+  }
+  return off;
+}
+
+pl_status validate_config(const pl_config* c) {
+  if (!c) return PL_EINVAL;
+  if (c->latent_c < 1 || c->latent_h < 1 || c->latent_w < 1) return PL_EINVAL;
+  if ((static_cast<int64_t>(c->latent_c) * c->latent_h * c->latent_w) % 4) return PL_EINVAL;
+  if (c->n_layers < 0 || c->n_layers > PL_MAX_LAYERS) return PL_EINVAL;
+  if (c->heads < 1) return PL_EINVAL;
+  if (c->append_cap < 0 || c->append_cap > PL_MAX_BANK - 1) return PL_EINVAL;
+  if (!(c->drift_threshold >= 0.f) || !std::isfinite(c->drift_threshold)) return PL_EINVAL;
+  for (int l = 0; l < c->n_layers; ++l) {
+    const int N = c->layer_tokens[l], C = c->layer_channels[l];
+    if (N < 1 || C < 1 || C % c->heads || C % 16) return PL_EINVAL;
+    if (!head_dim_supported(C / c->heads)) return PL_EUNSUPPORTED;
+  }
+  return PL_OK;
+}
+
+// Grouped K/V projection of bank features into entry `entry` of every layer.
+pl_status project_bank(pl_ctx* ctx, const void* const* feats, int entry, const int32_t* pred,
+                       cudaStream_t s) {
+  GemmParams gp;
+  std::memset(&gp, 0, sizeof(gp));
+  gp.status = &ctx->st->status;
+  int np = 0;
+  for (int l = 0; l < ctx->cfg.n_layers; ++l) {
+    if (!feats[l]) return PL_EINVAL;
+    const int N = ctx->cfg.layer_tokens[l], C = ctx->cfg.layer_channels[l];
+    const __half* wkv = static_cast<const __half*>(ctx->w[l].w_qkv) + C;
+    __half* dst = ctx->bank_kv[l] + static_cast<int64_t>(entry) * N * 2 * C;
+    const int r = pl::gemm_make_problem(&gp.prob[np], feats[l], C, wkv, 3 * C, dst, 2 * C, N,
+                                        2 * C, C, pred);
+    if (r) return gemm_status(r);
+    ++np;
+  }
+  gp.n_problems = np;
+  if (np == 0) return PL_OK;
+  return gemm_status(pl::gemm_launch(&gp, s, num_sms()));
+}
+
+pl_status single_gemm(const void* a, int64_t lda, const void* b, int64_t ldb, void* c,
+                      int64_t ldc, int M, int N, int K, uint32_t* status, cudaStream_t s) {
+  GemmParams gp;
+  std::memset(&gp, 0, sizeof(gp));
+  gp.status = status;
+  const int r = pl::gemm_make_problem(&gp.prob[0], a, lda, b, ldb, c, ldc, M, N, K, nullptr);
+  if (r) return gemm_status(r);
+  gp.n_problems = 1;
+  return gemm_status(pl::gemm_launch(&gp, s, num_sms()));
+}
+
+struct RoundArgs {
+  const float* new_noise;
+  const float* new_motion;
+  const void* const* hidden;
+  const float* eps;
+  float* out_frames;
+  uint8_t* appended;
+  void* const* layer_out;
+};
+
+// Enqueue one whole round on `s` (also used under stream capture).
+pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
+  const pl_config& c = ctx->cfg;
+  pl_status r = from_cuda(pl::launch_ring_push(ctx->st, ctx->ring, ctx->slot_motion,
+                                               ctx->batch_motion, a.new_noise, a.new_motion,
+                                               ctx->frame_elems, s));
+  if (r) return r;
+  for (int l = 0; l < c.n_layers; ++l) {
+    const int N = c.layer_tokens[l], C = c.layer_channels[l], H = c.heads, hd = C / H;
+    const int64_t M = 16ll * N;
+    const pl_layer_weights& w = ctx->w[l];
+    __half* out = a.layer_out ? static_cast<__half*>(a.layer_out[l]) : ctx->out_default;
+    r = from_cuda(pl::launch_motion_kv(ctx->batch_motion, static_cast<const __half*>(w.m_kv), 16,
+                                       C, ctx->tokens, ctx->motion_kv[l], s));
+    if (r) return r;
+    r = single_gemm(a.hidden[l], C, w.w_qkv, 3 * C, ctx->qkv, 3 * C, static_cast<int>(M), 3 * C,
+                    C, &ctx->st->status, s);
+    if (r) return r;
+    AttnSegHost segs[1 + PL_MAX_BANK];
+    segs[0] = {ctx->qkv + C, ctx->qkv + 2 * C, N, 3ll * C, static_cast<int64_t>(N) * 3 * C};
+    const int nb = ctx->have_anchors ? ctx->capacity : 1;
+    for (int b = 0; b < nb; ++b) {
+      const __half* kv = ctx->bank_kv[l] + static_cast<int64_t>(b) * N * 2 * C;
+      segs[1 + b] = {kv, kv + C, N, 2ll * C, 0};
+    }
+    AttnParams ap;
+    int ar = pl::attn_make_params(&ap, ctx->qkv, 3ll * C, static_cast<int64_t>(N) * 3 * C, segs,
+                                  1 + nb, 16, N, H, hd, ctx->attn_o, C,
+                                  static_cast<int64_t>(N) * C);
+    if (ar) return ar == 1 ? PL_EINVAL : PL_ECUDA;
+    ap.n_fixed = 2;
+    ap.n_extra = ctx->have_anchors ? &ctx->st->appends : nullptr;
+    ap.status = &ctx->st->status;
+    ar = pl::attn_launch(ap, hd, s);
+    if (ar) return ar == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
+    r = single_gemm(ctx->attn_o, C, w.w_o, C, ctx->a1, C, static_cast<int>(M), C, C,
+                    &ctx->st->status, s);
+    if (r) return r;
+    r = single_gemm(ctx->a1, C, w.m_q, C, ctx->qm, C, static_cast<int>(M), C, C,
+                    &ctx->st->status, s);
+    if (r) return r;
+    r = from_cuda(pl::launch_motion_attn(ctx->qm, C, ctx->motion_kv[l], 16, N, C, H, ctx->om, C, s));
+    if (r) return r;
+    r = single_gemm(ctx->om, C, w.m_o, C, out, C, static_cast<int>(M), C, C, &ctx->st->status, s);
+    if (r) return r;
+  }
+  r = from_cuda(pl::launch_ddim(ctx->st, ctx->ring, a.eps, a.out_frames, ctx->frame_elems,
+                                ctx->coef, s));
+  if (r) return r;
+  r = from_cuda(pl::launch_ring_commit(ctx->st, s));
+  if (r) return r;
+  r = from_cuda(pl::launch_bank_check(ctx->bank, &ctx->st->bank_count, &ctx->st->appends,
+                                      ctx->capacity, 512, a.new_motion, 4,
+                                      static_cast<double>(c.drift_threshold) * c.drift_threshold,
+                                      c.append_cap, nullptr, nullptr, a.appended, ctx->st, s));
+  if (r) return r;
+  if (ctx->have_anchors) {
+    for (int an = 1; an <= c.append_cap; ++an) {
+      r = project_bank(ctx, ctx->anchor_feats[an - 1], an, &ctx->st->anchor_fire[an], s);
+      if (r) return r;
+    }
+  }
+  return PL_OK;
+}
+
+void drop_graph(pl_ctx* ctx) {
+  if (ctx->exec) cudaGraphExecDestroy(ctx->exec);
+  if (ctx->graph) cudaGraphDestroy(ctx->graph);
+  ctx->exec = nullptr;
+  ctx->graph = nullptr;
+  ctx->key_n = 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pl_status_string(int status) {
+  switch (status) {
+    case PL_OK: return "ok";
+    case PL_EINVAL: return "invalid argument";
+    case PL_ESTATE: return "invalid state (call order)";
+    case PL_ENOMEM: return "workspace too small";
+    case PL_ECUDA: return "CUDA error";
+    case PL_ETIMEOUT: return "device wait timed out";
+    case PL_EDEVICE: return "device-side contract violation";
+    case PL_EUNSUPPORTED: return "unsupported shape";
+    default: return "unknown status";
+  }
+}
+
+int pl_abi_version(void) { return 1; }
+
+pl_status pl_gemm_f16(const void* a, int64_t lda, const void* b, int64_t ldb, void* c,
+                      int64_t ldc, int M, int N, int K, void* stream) {
+  if (!a || !b || !c) return PL_EINVAL;
+  return single_gemm(a, lda, b, ldb, c, ldc, M, N, K, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+pl_status pl_segment_attention(const void* q, int64_t ldq, int64_t q_frame_stride,
+                               const pl_kv_segment* segs, int n_segs, int frames, int n_q,
+                               int heads, int head_dim, void* out, int64_t ldo,
+                               int64_t out_frame_stride, void* stream) {
+  if (!q || !segs || !out) return PL_EINVAL;
+  if (n_segs < 1 || n_segs > pl::kAttnMaxSegs) return PL_EINVAL;
+  if (!head_dim_supported(head_dim)) return PL_EUNSUPPORTED;
+  if (frames > 65535 || heads > 65535) return PL_EINVAL;
+  AttnSegHost hs[pl::kAttnMaxSegs];
+  for (int i = 0; i < n_segs; ++i) {
+    if (!segs[i].k || !segs[i].v) return PL_EINVAL;
+    hs[i] = {segs[i].k, segs[i].v, segs[i].len, segs[i].ld, segs[i].frame_stride};
+  }
+  AttnParams p;
+  const int r = pl::attn_make_params(&p, q, ldq, q_frame_stride, hs, n_segs, frames, n_q, heads,
+                                     head_dim, out, ldo, out_frame_stride);
+  if (r) return r == 1 ? PL_EINVAL : PL_ECUDA;
+  const int lr = pl::attn_launch(p, head_dim, static_cast<cudaStream_t>(stream));
+  return lr == 0 ? PL_OK : lr == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
+}
+
+pl_status pl_ref_attention_workspace_bytes(int frames, int n, int c, int n_bank, size_t* bytes) {
+  if (!bytes || frames < 1 || n < 1 || c < 1 || n_bank < 0 || n_bank > PL_MAX_BANK)
+    return PL_EINVAL;
+  const size_t fnc = static_cast<size_t>(frames) * n * c;
+  *bytes = align_up(2 * 3 * fnc) + align_up(2 * static_cast<size_t>(n_bank) * n * 2 * c) +
+           align_up(2 * fnc);
+  return PL_OK;
+}
+
+pl_status pl_ref_attention(const void* hidden, const void* w_qkv, const void* w_o,
+                           const void* const* bank_feats, int n_bank, int frames, int n, int c,
+                           int heads, void* out, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (!hidden || !w_qkv || !w_o || !out || !workspace) return PL_EINVAL;
+  if (heads < 1 || c % heads || c % 16) return PL_EINVAL;
+  if (n_bank < 0 || n_bank > PL_MAX_BANK || (n_bank > 0 && !bank_feats)) return PL_EINVAL;
+  const int hd = c / heads;
+  if (!head_dim_supported(hd)) return PL_EUNSUPPORTED;
+  size_t need = 0;
+  if (pl_ref_attention_workspace_bytes(frames, n, c, n_bank, &need)) return PL_EINVAL;
+  if (workspace_bytes < need) return PL_ENOMEM;
+  if (!aligned16(workspace)) return PL_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t fnc = static_cast<size_t>(frames) * n * c;
+  __half* qkv = static_cast<__half*>(workspace);
+  __half* bkv = reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(workspace) +
+                                          align_up(2 * 3 * fnc));
+  __half* o = reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(bkv) +
+                                        align_up(2 * static_cast<size_t>(n_bank) * n * 2 * c));
+  GemmParams gp;
+  std::memset(&gp, 0, sizeof(gp));
+  int r = pl::gemm_make_problem(&gp.prob[0], hidden, c, w_qkv, 3 * c, qkv, 3 * c, frames * n,
+                                3 * c, c, nullptr);
+  if (r) return gemm_status(r);
+  for (int b = 0; b < n_bank; ++b) {
+    if (!bank_feats[b]) return PL_EINVAL;
+    r = pl::gemm_make_problem(&gp.prob[1 + b], bank_feats[b], c,
+                              static_cast<const __half*>(w_qkv) + c, 3 * c,
+                              bkv + static_cast<int64_t>(b) * n * 2 * c, 2 * c, n, 2 * c, c,
+                              nullptr);
+    if (r) return gemm_status(r);
+  }
+  gp.n_problems = 1 + n_bank;
+  r = pl::gemm_launch(&gp, s, num_sms());
+  if (r) return gemm_status(r);
+  AttnSegHost segs[1 + PL_MAX_BANK];
+  segs[0] = {qkv + c, qkv + 2 * c, n, 3ll * c, static_cast<int64_t>(n) * 3 * c};
+  for (int b = 0; b < n_bank; ++b) {
+    const __half* kv = bkv + static_cast<int64_t>(b) * n * 2 * c;
+    segs[1 + b] = {kv, kv + c, n, 2ll * c, 0};
+  }
+  AttnParams ap;
+  r = pl::attn_make_params(&ap, qkv, 3ll * c, static_cast<int64_t>(n) * 3 * c, segs, 1 + n_bank,
+                           frames, n, heads, hd, o, c, static_cast<int64_t>(n) * c);
+  if (r) return r == 1 ? PL_EINVAL : PL_ECUDA;
+  r = pl::attn_launch(ap, hd, s);
+  if (r) return r == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
+  return single_gemm(o, c, w_o, c, out, c, frames * n, c, c, nullptr, s);
+}
+
+pl_status pl_motion_xattn_workspace_bytes(int frames, int n, int c, size_t* bytes) {
+  if (!bytes || frames < 1 || n < 1 || c < 1) return PL_EINVAL;
+  const size_t fnc = static_cast<size_t>(frames) * n * c;
+  *bytes = align_up(2 * static_cast<size_t>(frames) * 512) +
+           align_up(2 * static_cast<size_t>(frames) * 32 * 2 * c) + 2 * align_up(2 * fnc);
+  return PL_OK;
+}
+
+pl_status pl_motion_xattn(const void* x, const float* motion, const void* m_q, const void* m_kv,
+                          const void* m_o, int frames, int n, int c, int heads, void* out,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x || !motion || !m_q || !m_kv || !m_o || !out || !workspace) return PL_EINVAL;
+  if (heads < 1 || c % heads || c % 16 || frames < 1 || frames > 65535 || n < 1) return PL_EINVAL;
+  if (!head_dim_supported(c / heads)) return PL_EUNSUPPORTED;
+  size_t need = 0;
+  if (pl_motion_xattn_workspace_bytes(frames, n, c, &need)) return PL_EINVAL;
+  if (workspace_bytes < need) return PL_ENOMEM;
+  if (!aligned16(workspace)) return PL_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t fnc = static_cast<size_t>(frames) * n * c;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  __half* tok = reinterpret_cast<__half*>(w);
+  w += align_up(2 * static_cast<size_t>(frames) * 512);
+  __half* kv = reinterpret_cast<__half*>(w);
+  w += align_up(2 * static_cast<size_t>(frames) * 32 * 2 * c);
+  __half* qm = reinterpret_cast<__half*>(w);
+  w += align_up(2 * fnc);
+  __half* om = reinterpret_cast<__half*>(w);
+  pl_status r = from_cuda(pl::launch_motion_kv(motion, static_cast<const __half*>(m_kv), frames,
+                                               c, tok, kv, s));
+  if (r) return r;
+  r = single_gemm(x, c, m_q, c, qm, c, frames * n, c, c, nullptr, s);
+  if (r) return r;
+  r = from_cuda(pl::launch_motion_attn(qm, c, kv, frames, n, c, heads, om, c, s));
+  if (r) return r;
+  return single_gemm(om, c, m_o, c, out, c, frames * n, c, c, nullptr, s);
+}
+
+pl_status pl_motion_bank_check(float* bank, int32_t* count, int32_t* appends, int capacity,
+                               int dim, const float* queries, int n_queries, float threshold,
+                               int cap, int32_t* argmin, double* min_d2, uint8_t* appended,
+                               void* stream) {
+  if (!bank || !count || !appends || (n_queries > 0 && !queries)) return PL_EINVAL;
+  if (dim < 1 || dim > 4096 || capacity < 1 || capacity > 65536) return PL_EINVAL;
+  if (n_queries < 0 || n_queries > 64 || cap < 0) return PL_EINVAL;
+  if (!(threshold >= 0.f) || !std::isfinite(threshold)) return PL_EINVAL;
+  if (n_queries == 0) return PL_OK;
+  const double thr2 = static_cast<double>(threshold) * threshold;
+  return from_cuda(pl::launch_bank_check(bank, count, appends, capacity, dim, queries, n_queries,
+                                         thr2, cap, argmin, min_d2, appended, nullptr,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+pl_status pl_workspace_bytes(const pl_config* cfg, size_t* bytes) {
+  if (!bytes) return PL_EINVAL;
+  const pl_status v = validate_config(cfg);
+  if (v) return v;
+  *bytes = layout(*cfg, nullptr);
+  return PL_OK;
+}
+
+pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_bytes,
+                        pl_ctx** out) {
+  if (!out || !workspace) return PL_EINVAL;
+  *out = nullptr;
+  const pl_status v = validate_config(cfg);
+  if (v) return v;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return PL_EINVAL;
+  const size_t need = layout(*cfg, nullptr);
+  if (workspace_bytes < need) return PL_ENOMEM;
+  pl_ctx* ctx = new (std::nothrow) pl_ctx;
+  if (!ctx) return PL_ENOMEM;
+  std::memset(static_cast<void*>(ctx), 0, sizeof(*ctx));
+  ctx->cfg = *cfg;
+  ctx->capacity = 1 + cfg->append_cap;
+  ctx->frame_elems = static_cast<int64_t>(cfg->latent_c) * cfg->latent_h * cfg->latent_w;
+  ctx->ws = static_cast<uint8_t*>(workspace);
+  ctx->ws_bytes = workspace_bytes;
+  layout(*cfg, ctx);
+  pl::ddim_coefficients(&ctx->coef);
+  // zero the device state so pl_get_state is meaningful before bank_init
+  if (cudaMemset(ctx->st, 0, sizeof(pl::DevState)) != cudaSuccess) {
+    delete ctx;
+    return PL_ECUDA;
+  }
+  *out = ctx;
+  return PL_OK;
+}
+
+pl_status pl_ctx_destroy(pl_ctx* ctx) {
+  if (!ctx) return PL_OK;
+  drop_graph(ctx);
+  delete ctx;
+  return PL_OK;
+}
+
+pl_status pl_bank_init(pl_ctx* ctx, const pl_layer_weights* weights,
+                       const void* const* ref_feats, const void* const* anchor_feats,
+                       const float* ref_motion, const float* drive0_motion,
+                       const float* ref_latent, const float* prefill_eps, void* stream) {
+  if (!ctx || !ref_motion || !drive0_motion || !ref_latent || !prefill_eps) return PL_EINVAL;
+  const int L = ctx->cfg.n_layers;
+  if (L > 0 && (!weights || !ref_feats)) return PL_EINVAL;
+  for (int l = 0; l < L; ++l) {
+    const pl_layer_weights& w = weights[l];
+    if (!w.w_qkv || !w.w_o || !w.m_q || !w.m_kv || !w.m_o || !ref_feats[l]) return PL_EINVAL;
+    ctx->w[l] = w;
+    ctx->ref_feats[l] = ref_feats[l];
+  }
+  ctx->have_anchors = anchor_feats != nullptr && L > 0 && ctx->cfg.append_cap > 0;
+  if (ctx->have_anchors) {
+    for (int a = 0; a < ctx->cfg.append_cap; ++a)
+      for (int l = 0; l < L; ++l) {
+        ctx->anchor_feats[a][l] = anchor_feats[a * L + l];
+        if (!ctx->anchor_feats[a][l]) return PL_EINVAL;
+      }
+  }
+  drop_graph(ctx);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  pl_status r = from_cuda(pl::launch_prefill(ctx->st, ctx->ring, ctx->slot_motion, ctx->bank,
+                                             ref_latent, prefill_eps, ref_motion, drive0_motion,
+                                             ctx->frame_elems, s));
+  if (r) return r;
+  if (L > 0) {
+    r = project_bank(ctx, ctx->ref_feats, 0, nullptr, s);
+    if (r) return r;
+  }
+  ctx->initialised = true;
+  return PL_OK;
+}
+
+pl_status pl_ring_push(pl_ctx* ctx, const float* new_noise, const float* new_motion,
+                       void* stream) {
+  if (!ctx || !new_noise || !new_motion) return PL_EINVAL;
+  if (!ctx->initialised) return PL_ESTATE;
+  return from_cuda(pl::launch_ring_push(ctx->st, ctx->ring, ctx->slot_motion, ctx->batch_motion,
+                                        new_noise, new_motion, ctx->frame_elems,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+pl_status pl_pyramid_ddim_step(pl_ctx* ctx, const float* eps, float* out_x0, void* stream) {
+  if (!ctx || !eps || !out_x0) return PL_EINVAL;
+  if (!ctx->initialised) return PL_ESTATE;
+  if (!aligned16(eps) || !aligned16(out_x0)) return PL_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  pl_status r = from_cuda(pl::launch_ddim(ctx->st, ctx->ring, eps, out_x0, ctx->frame_elems,
+                                          ctx->coef, s));
+  if (r) return r;
+  return from_cuda(pl::launch_ring_commit(ctx->st, s));
+}
+
+pl_status pl_ctx_bank_check(pl_ctx* ctx, const float* queries, int n_queries, int32_t* argmin,
+                            double* min_d2, uint8_t* appended, void* stream) {
+  if (!ctx || (n_queries > 0 && !queries) || n_queries < 0 || n_queries > 64) return PL_EINVAL;
+  if (!ctx->initialised) return PL_ESTATE;
+  if (n_queries == 0) return PL_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const pl_config& c = ctx->cfg;
+  pl_status r = from_cuda(pl::launch_bank_check(
+      ctx->bank, &ctx->st->bank_count, &ctx->st->appends, ctx->capacity, 512, queries, n_queries,
+      static_cast<double>(c.drift_threshold) * c.drift_threshold, c.append_cap, argmin, min_d2,
+      appended, ctx->st, s));
+  if (r) return r;
+  if (ctx->have_anchors) {
+    for (int an = 1; an <= c.append_cap; ++an) {
+      r = project_bank(ctx, ctx->anchor_feats[an - 1], an, &ctx->st->anchor_fire[an], s);
+      if (r) return r;
+    }
+  }
+  return PL_OK;
+}
+
+pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_motion,
+                          const void* const* hidden, const float* eps, float* out_frames,
+                          uint8_t* appended, void* const* layer_out, void* stream) {
+  if (!ctx || !new_noise || !new_motion || !eps || !out_frames) return PL_EINVAL;
+  if (!ctx->initialised) return PL_ESTATE;
+  const int L = ctx->cfg.n_layers;
+  if (L > 0 && !hidden) return PL_EINVAL;
+  for (int l = 0; l < L; ++l) {
+    if (!hidden[l] || !aligned16(hidden[l])) return PL_EINVAL;
+    if (layer_out && (!layer_out[l] || !aligned16(layer_out[l]))) return PL_EINVAL;
+  }
+  if (!aligned16(new_noise) || !aligned16(eps) || !aligned16(out_frames)) return PL_EINVAL;
+  RoundArgs a{new_noise, new_motion, hidden, eps, out_frames, appended, layer_out};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const char* env = std::getenv("PL_NO_GRAPH");
+  const bool use_graph = s != nullptr && !(env && env[0] == '1');
+  if (!use_graph) return enqueue_round(ctx, a, s);
+  // key = every pointer the captured launches bake in
+  const void* key[64];
+  int kn = 0;
+  key[kn++] = new_noise;
+  key[kn++] = new_motion;
+  key[kn++] = eps;
+  key[kn++] = out_frames;
+  key[kn++] = appended;
+  key[kn++] = layer_out ? reinterpret_cast<const void*>(1) : nullptr;
+  for (int l = 0; l < L; ++l) {
+    key[kn++] = hidden[l];
+    key[kn++] = layer_out ? layer_out[l] : nullptr;
+  }
+  bool hit = ctx->exec && ctx->key_n == kn;
+  for (int i = 0; hit && i < kn; ++i) hit = ctx->key[i] == key[i];
+  if (!hit) {
+    drop_graph(ctx);
+    if (cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+      return PL_ECUDA;
+    const pl_status r = enqueue_round(ctx, a, s);
+    cudaGraph_t g = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(s, &g);
+    if (r != PL_OK) {
+      if (g) cudaGraphDestroy(g);
+      return r;
+    }
+    if (e != cudaSuccess || !g) return PL_ECUDA;
+    if (cudaGraphInstantiate(&ctx->exec, g, 0) != cudaSuccess) {
+      cudaGraphDestroy(g);
+      ctx->exec = nullptr;
+      return PL_ECUDA;
+    }
+    ctx->graph = g;
+    std::memcpy(ctx->key, key, sizeof(const void*) * kn);
+    ctx->key_n = kn;
+  }
+  return from_cuda(cudaGraphLaunch(ctx->exec, s));
+}
+
+pl_status pl_get_state(pl_ctx* ctx, pl_state* out, void* stream) {
+  if (!ctx || !out) return PL_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PL_ECUDA;
+  pl::DevState d;
+  if (cudaMemcpy(&d, ctx->st, sizeof(d), cudaMemcpyDeviceToHost) != cudaSuccess) return PL_ECUDA;
+  std::memset(out, 0, sizeof(*out));
+  out->initialised = ctx->initialised ? d.initialised : 0;
+  out->head = d.head;
+  for (int i = 0; i < 4; ++i) out->slot_t[i] = d.slot_t[i];
+  out->rounds = d.rounds;
+  out->frames_in = d.frames_in;
+  out->frames_out = d.frames_out;
+  out->bank_count = d.bank_count;
+  out->appends = d.appends;
+  out->device_status = d.status;
+  return PL_OK;
+}
+
+pl_status pl_get_motion_bank(pl_ctx* ctx, float* host_out, int32_t* count, void* stream) {
+  if (!ctx || !host_out || !count) return PL_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PL_ECUDA;
+  int32_t n = 0;
+  if (cudaMemcpy(&n, &ctx->st->bank_count, sizeof(n), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return PL_ECUDA;
+  if (n < 0 || n > ctx->capacity) return PL_EDEVICE;
+  *count = n;
+  if (n > 0 && cudaMemcpy(host_out, ctx->bank, sizeof(float) * 512 * n, cudaMemcpyDeviceToHost) !=
+                   cudaSuccess)
+    return PL_ECUDA;
+  return PL_OK;
+}
+
+pl_status pl_get_device_status(pl_ctx* ctx, void* stream) {
+  if (!ctx) return PL_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PL_ECUDA;
+  uint32_t w = 0;
+  if (cudaMemcpy(&w, &ctx->st->status, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return PL_ECUDA;
+  const uint32_t zero = 0;
+  if (cudaMemcpy(&ctx->st->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+    return PL_ECUDA;
+  if (w & pl::DEV_TIMEOUT) return PL_ETIMEOUT;
+  if (w) return PL_EDEVICE;
+  return PL_OK;
+}
+
+const float* pl_ctx_ring_latents(const pl_ctx* ctx) { return ctx ? ctx->ring : nullptr; }
+
+}  // extern "C"

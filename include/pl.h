@@ -1,0 +1,273 @@
+/*
+ * pl.h — C ABI of the streaming pyramid denoising round (PersonaLive) on B200.
+ *
+ * One round, as the PersonaLive write-up (juhe.plus) describes it in
+ * "流式金字塔去噪" (streaming pyramid denoising): a pile of 4 windows x 4
+ * latent frames sits at DDIM timesteps {999, 666, 333, 0}; each round appends
+ * a new noise window at t = 999, runs the 16 frames as one batch, moves every
+ * window one DDIM step (step length 333) and pops the t = 0 window with its
+ * predicted x0. Inside the batch every reference-attention layer attends over
+ * the frame's own tokens concatenated with a reference KV bank of 1..4 entries
+ * ("三条条件通路", three conditioning paths), next to a 32-token, 16-d motion
+ * cross-attention. After the step the round's motion embeddings are checked
+ * against a motion bank (minimum L2 distance > 17 appends an anchor, at most 3
+ * times; "抗身份漂移的补丁", identity-drift guard).
+ *
+ * Conventions for every call:
+ *  - Pointers named as device pointers must point to memory of the current
+ *    CUDA device; the caller allocates and owns all of it (the library never
+ *    allocates device memory). Host pointers are read before the call returns.
+ *  - All fp16 matrices are row-major with the stated leading dimension in
+ *    ELEMENTS; leading dimensions and frame strides must be multiples of 8
+ *    (16 bytes) and device pointers 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Every call is
+ *    asynchronous on it unless stated otherwise.
+ *  - The return value reports host-side validation and launch errors only.
+ *    Kernels that detect a problem on the device (a bounded wait that ran
+ *    out, an argument outside the contract) set bits of a device status word
+ *    instead of trapping; read it with pl_get_device_status().
+ *  - Nothing aborts, exits or traps. A context is not thread-safe.
+ */
+#ifndef PL_H_
+#define PL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pl_status {
+  PL_OK = 0,
+  PL_EINVAL = 1,       /* an argument is outside its documented range */
+  PL_ESTATE = 2,       /* call order violated (e.g. a round before pl_bank_init) */
+  PL_ENOMEM = 3,       /* the caller's workspace is smaller than required */
+  PL_ECUDA = 4,        /* a CUDA runtime/driver call failed */
+  PL_ETIMEOUT = 5,     /* a device-side bounded wait gave up */
+  PL_EDEVICE = 6,      /* a kernel flagged a contract violation on the device */
+  PL_EUNSUPPORTED = 7  /* shape not supported by this build (e.g. head_dim) */
+} pl_status;
+
+/* Static description of a status code. Never NULL. */
+const char* pl_status_string(int status);
+
+/* ABI version of this header (incremented on any signature change). */
+int pl_abi_version(void);
+
+/* ------------------------------------------------------------------ *
+ * Stateless primitives
+ * ------------------------------------------------------------------ */
+
+/* C[M,N] = A[M,K] * B[K,N] (fp16 in, fp32 accumulate, fp16 out) on tcgen05
+ * tensor cores. a, b, c: device pointers; lda >= K, ldb >= N, ldc >= N.
+ * Requires N % 16 == 0 and K % 8 == 0. Used for every projection of the
+ * reference attention (Q/K/V/O) and of the motion cross-attention (Q/O). */
+pl_status pl_gemm_f16(const void* a, int64_t lda, const void* b, int64_t ldb, void* c,
+                      int64_t ldc, int M, int N, int K, void* stream);
+
+/* One KV segment of an attention call. Row r of frame f of the segment's K
+ * starts at element (f * frame_stride + r) * ld of `k` (same for `v`); head h
+ * occupies columns [h * head_dim, (h + 1) * head_dim). frame_stride == 0
+ * means the segment is shared by all frames (a reference bank entry). */
+typedef struct pl_kv_segment {
+  const void* k;          /* device, fp16 */
+  const void* v;          /* device, fp16 */
+  int64_t len;            /* rows (keys) in the segment, >= 1 */
+  int64_t ld;             /* elements between rows, multiple of 8 */
+  int64_t frame_stride;   /* elements between frames, multiple of 8, or 0 */
+} pl_kv_segment;
+
+/* Attention core over a list of KV segments, never materialising their
+ * concatenation (PersonaLive write-up, "三条条件通路": own KV followed by the
+ * reference bank; LiveAnimate page, PR-Sink: query block + sink + retrieved
+ * block + rolling blocks):
+ *   out[f, i, h] = softmax_j( q[f,i,h] . K_cat[f,j,h] / sqrt(head_dim) ) V_cat[f,j,h]
+ * with K_cat/V_cat = segments in order. Full (non-causal) attention, fp32
+ * softmax statistics, fp16 output.
+ * q: device [frames][n_q][ldq] (frame stride q_frame_stride elements);
+ * out: device, same addressing with ldo / out_frame_stride.
+ * head_dim in {40, 64, 80, 128, 160}; 1 <= n_segs <= 8. */
+pl_status pl_segment_attention(const void* q, int64_t ldq, int64_t q_frame_stride,
+                               const pl_kv_segment* segs, int n_segs, int frames, int n_q,
+                               int heads, int head_dim, void* out, int64_t ldo,
+                               int64_t out_frame_stride, void* stream);
+
+/* Bytes of device workspace pl_ref_attention needs. */
+pl_status pl_ref_attention_workspace_bytes(int frames, int n, int c, int n_bank,
+                                           size_t* bytes);
+
+/* One reference-attention layer (PersonaLive write-up, "三条条件通路"):
+ *   Q = h Wq; K = [h ; bank_0 ; ...] Wk; V = [h ; bank_0 ; ...] Wv;
+ *   out = attention(Q, K, V) Wo,  8-head split of C, scale 1/sqrt(C/heads).
+ * hidden: device fp16 [frames][n][c]; w_qkv: device fp16 [c][3c] = [Wq|Wk|Wv];
+ * w_o: device fp16 [c][c]; bank_feats: host array of n_bank device pointers,
+ * each fp16 [n][c] (norm_hidden_states of the Reference UNet, shared by all
+ * frames); out: device fp16 [frames][n][c]. 0 <= n_bank <= 4.
+ * workspace: device, >= pl_ref_attention_workspace_bytes(). */
+pl_status pl_ref_attention(const void* hidden, const void* w_qkv, const void* w_o,
+                           const void* const* bank_feats, int n_bank, int frames, int n,
+                           int c, int heads, void* out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace pl_motion_xattn needs. */
+pl_status pl_motion_xattn_workspace_bytes(int frames, int n, int c, size_t* bytes);
+
+/* Motion cross-attention (PersonaLive write-up, "三条条件通路": the 512-d
+ * expression embedding becomes 32 tokens x 16 channels plus a sinusoidal
+ * position code; cross_attention_dim 16; 8 heads):
+ *   tok[f] = reshape(motion[f], 32, 16) + PE  (PE[p,2i] = sin(p/10000^(2i/16)),
+ *            PE[p,2i+1] = cos(same)), rounded to fp16;
+ *   out = softmax((x Mq)(tok Mk)^T / sqrt(c/heads)) (tok Mv) Mo.
+ * x: device fp16 [frames][n][c]; motion: device fp32 [frames][512];
+ * m_q, m_o: device fp16 [c][c]; m_kv: device fp16 [16][2c] = [Mk|Mv];
+ * out: device fp16 [frames][n][c]. */
+pl_status pl_motion_xattn(const void* x, const float* motion, const void* m_q,
+                          const void* m_kv, const void* m_o, int frames, int n, int c,
+                          int heads, void* out, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* Motion-bank check (PersonaLive write-up, "抗身份漂移的补丁"), in query
+ * order: for query q, d2_j = ||q - bank_j||^2 (fp64) over the *count entries
+ * present (including entries appended earlier in this call); argmin = lowest
+ * index of the minimum; if d2_min > threshold^2 and *appends < cap and
+ * *count < capacity, q is copied to bank[*count], ++*count, ++*appends.
+ * bank: device fp32 [capacity][dim]; count, appends: device int32 (state,
+ * read and updated on the device); queries: device fp32 [n_queries][dim];
+ * argmin (int32), min_d2 (double), appended (uint8): device [n_queries],
+ * each may be NULL. cap = 0 turns the call into a pure nearest-neighbour
+ * retrieval (LiveAnimate page, PR-Sink's pose-retrieved dynamic sink).
+ * 1 <= dim <= 4096, 1 <= capacity <= 65536, 0 <= n_queries <= 64. */
+pl_status pl_motion_bank_check(float* bank, int32_t* count, int32_t* appends, int capacity,
+                               int dim, const float* queries, int n_queries, float threshold,
+                               int cap, int32_t* argmin, double* min_d2, uint8_t* appended,
+                               void* stream);
+
+/* ------------------------------------------------------------------ *
+ * Stream context: the device-resident pile and the reference bank
+ * ------------------------------------------------------------------ */
+
+typedef struct pl_ctx pl_ctx;
+
+#define PL_MAX_LAYERS 16
+#define PL_WINDOWS 4            /* temporal_adaptive_step */
+#define PL_WINDOW_FRAMES 4      /* temporal_window_size */
+#define PL_BATCH_FRAMES 16
+#define PL_MOTION_DIM 512
+#define PL_MAX_BANK 4           /* reference + up to 3 anchors */
+
+typedef struct pl_config {
+  int32_t latent_c;                      /* 4 */
+  int32_t latent_h, latent_w;            /* 64 x 64 for 512 x 512 frames */
+  int32_t n_layers;                      /* 0..16 reference-attention layers */
+  int32_t layer_tokens[PL_MAX_LAYERS];   /* tokens per frame N_l */
+  int32_t layer_channels[PL_MAX_LAYERS]; /* channels C_l (multiple of heads*8) */
+  int32_t heads;                         /* 8 */
+  float drift_threshold;                 /* 17 */
+  int32_t append_cap;                    /* 3 (so the bank holds at most 4) */
+} pl_config;
+
+/* Per-layer weights (device fp16, row-major [in][out]); kept by pointer, so
+ * they must outlive the context. */
+typedef struct pl_layer_weights {
+  const void* w_qkv; /* [C][3C] = [Wq | Wk | Wv] */
+  const void* w_o;   /* [C][C] */
+  const void* m_q;   /* [C][C] motion query projection */
+  const void* m_kv;  /* [16][2C] = [Mk | Mv] */
+  const void* m_o;   /* [C][C] */
+} pl_layer_weights;
+
+/* Host-side snapshot of the context's state (pl_get_state). */
+typedef struct pl_state {
+  int32_t initialised;
+  int32_t head;                 /* physical slot of the oldest window */
+  int32_t slot_t[PL_WINDOWS];   /* timestep per physical slot, -1 = free */
+  int64_t rounds;
+  int64_t frames_in;
+  int64_t frames_out;
+  int32_t bank_count;           /* entries in the motion bank == KV bank entries */
+  int32_t appends;              /* anchors appended so far (<= append_cap) */
+  uint32_t device_status;       /* bits set by kernels (0 = clean) */
+} pl_state;
+
+/* Device workspace a context with this configuration needs. */
+pl_status pl_workspace_bytes(const pl_config* cfg, size_t* bytes);
+
+/* Create a context on the current device inside the caller's workspace
+ * (device memory, >= pl_workspace_bytes, 256-byte aligned). The context
+ * struct itself lives in host memory owned by the library. */
+pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_bytes,
+                        pl_ctx** out);
+
+/* Destroy (releases host memory and any captured CUDA graph). NULL is a no-op. */
+pl_status pl_ctx_destroy(pl_ctx* ctx);
+
+/* Reference fusion, also the control-plane reset (PersonaLive write-up,
+ * "首帧怎么办" and the pause/reset remark of "在线链路"):
+ *  - KV bank <- entry 0 = ref_feats[l] projected by each layer's Wk/Wv;
+ *  - motion bank <- [ref_motion], appends <- 0;
+ *  - prefill: 3 windows at t = 0, 333, 666 (oldest first), window w frame j =
+ *    sqrt(abar_t) ref_latent + sqrt(1 - abar_t) prefill_eps[4w + j], with the
+ *    12 frames' motion = ref + (k/12)(drive0 - ref), k = 0..11.
+ * weights: host array [n_layers]; ref_feats: host array of n_layers device
+ * fp16 [N_l][C_l]; anchor_feats: host array of 3*n_layers device pointers
+ * (anchor a = 1..3, layer l at index (a-1)*n_layers + l) standing in for the
+ * Reference UNet re-run of an anchor frame, or NULL (then appends extend only
+ * the motion bank and the KV bank keeps entry 0). ref_motion, drive0_motion:
+ * device fp32 [512]; ref_latent: device fp32 [4][H][W]; prefill_eps: device
+ * fp32 [12][4][H][W]. All pointers must stay valid for the context's life. */
+pl_status pl_bank_init(pl_ctx* ctx, const pl_layer_weights* weights,
+                       const void* const* ref_feats, const void* const* anchor_feats,
+                       const float* ref_motion, const float* drive0_motion,
+                       const float* ref_latent, const float* prefill_eps, void* stream);
+
+/* Append the new window (pure noise at t = 999) into the free slot.
+ * new_noise: device fp32 [4][4][H][W]; new_motion: device fp32 [4][512]. */
+pl_status pl_ring_push(pl_ctx* ctx, const float* new_noise, const float* new_motion,
+                       void* stream);
+
+/* One DDIM step (eta = 0, epsilon prediction, SD scaled-linear betas
+ * 0.00085..0.012 over 1000 steps, step length 333) of every window of the
+ * full pile, then the pop: out_x0 <- x0 of the t = 0 window, its slot freed.
+ * eps: device fp32 [16][4][H][W] in batch order (oldest window first);
+ * out_x0: device fp32 [4][4][H][W]. Requires a full pile (after pl_ring_push). */
+pl_status pl_pyramid_ddim_step(pl_ctx* ctx, const float* eps, float* out_x0, void* stream);
+
+/* pl_motion_bank_check on the context's motion bank with its threshold and
+ * cap. When an append happens and anchor features were given, the anchor's
+ * K/V are projected for every layer into the next KV-bank entry. */
+pl_status pl_ctx_bank_check(pl_ctx* ctx, const float* queries, int n_queries,
+                            int32_t* argmin, double* min_d2, uint8_t* appended,
+                            void* stream);
+
+/* One whole round: ring push, the n_layers reference-attention + motion
+ * cross-attention layers on the 16-frame batch, the pyramid DDIM step with
+ * pop, and the bank check of the 4 new motion embeddings.
+ * hidden: host array [n_layers] of device fp16 [16][N_l][C_l] (batch order);
+ * eps: device fp32 [16][4][H][W]; out_frames: device fp32 [4][4][H][W];
+ * appended: device uint8 [4] or NULL; layer_out: host array [n_layers] of
+ * device fp16 [16][N_l][C_l] or NULL (outputs then go to workspace).
+ * The round is recorded as a CUDA graph on the first call and replayed while
+ * the pointer arguments stay the same. */
+pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_motion,
+                          const void* const* hidden, const float* eps, float* out_frames,
+                          uint8_t* appended, void* const* layer_out, void* stream);
+
+/* Synchronise `stream` and copy the context's state to *out. */
+pl_status pl_get_state(pl_ctx* ctx, pl_state* out, void* stream);
+
+/* Synchronise `stream`, copy the motion bank (fp32 [count][512]) to host. */
+pl_status pl_get_motion_bank(pl_ctx* ctx, float* host_out, int32_t* count, void* stream);
+
+/* Synchronise `stream` and map the device status word to a status:
+ * PL_OK, PL_ETIMEOUT or PL_EDEVICE. Clears the word. */
+pl_status pl_get_device_status(pl_ctx* ctx, void* stream);
+
+/* Device pointer of the pile's latents, fp32 [4 slots][4][4][H][W] (read-only
+ * view for tests; slot s holds the window at timestep slot_t[s]). */
+const float* pl_ctx_ring_latents(const pl_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PL_H_ */

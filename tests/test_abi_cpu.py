@@ -1,0 +1,80 @@
+"""The C-ABI library loads and exports every symbol include/pl.h declares, and
+its host-side validation rejects bad arguments without touching a GPU."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "pl.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pl_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary_calls():
+    names = _declared()
+    for must in ("pl_bank_init", "pl_ref_attention", "pl_motion_xattn", "pl_pyramid_ddim_step",
+                 "pl_motion_bank_check", "pl_stream_round"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    import denoise_step_b200 as P
+    for name in _declared():
+        assert hasattr(P.lib, name), name
+        assert name in P.EXPORTED, name
+
+
+def test_status_strings_and_abi():
+    import denoise_step_b200 as P
+    assert P.lib.pl_abi_version() == 1
+    for s in range(8):
+        assert P.lib.pl_status_string(s)
+    assert P.lib.pl_status_string(99) == b"unknown status"
+
+
+def test_host_validation_rejects_bad_arguments():
+    import denoise_step_b200 as P
+    L = P.lib
+    assert L.pl_gemm_f16(None, 8, None, 8, None, 8, 8, 16, 8, None) == P.PL_EINVAL
+    n = C.c_size_t()
+    assert L.pl_ref_attention_workspace_bytes(0, 64, 1280, 1, C.byref(n)) == P.PL_EINVAL
+    assert L.pl_ref_attention_workspace_bytes(16, 64, 1280, 5, C.byref(n)) == P.PL_EINVAL
+    assert L.pl_ref_attention_workspace_bytes(16, 64, 1280, 1, C.byref(n)) == P.PL_OK
+    # qkv 3*F*N*C + bank 2*N*C + o F*N*C halves, each region 256-byte aligned
+    assert n.value >= 2 * (3 * 16 * 64 * 1280 + 2 * 64 * 1280 + 16 * 64 * 1280)
+    seg = (P.KVSegment * 1)()
+    assert L.pl_segment_attention(None, 8, 8, seg, 1, 1, 1, 1, 40, None, 8, 8, None) == P.PL_EINVAL
+    assert L.pl_motion_bank_check(None, None, None, 4, 512, None, 1, 17.0, 3, None, None, None,
+                                  None) == P.PL_EINVAL
+    assert L.pl_ctx_destroy(None) == P.PL_OK
+
+
+def test_config_validation_and_workspace_size():
+    import denoise_step_b200 as P
+    import synthetic as S
+    layers = [(side * side, c) for _, side, c in S.LAYERS]
+    cfg = P.make_config((64, 64), layers)
+    n = C.c_size_t()
+    assert P.lib.pl_workspace_bytes(C.byref(cfg), C.byref(n)) == P.PL_OK
+    assert n.value > 0
+    bad = P.make_config((64, 64), [(4096, 320)], heads=7)
+    assert P.lib.pl_workspace_bytes(C.byref(bad), C.byref(n)) == P.PL_EINVAL
+    unsup = P.make_config((64, 64), [(4096, 96 * 8)], heads=8)        # head_dim 96
+    assert P.lib.pl_workspace_bytes(C.byref(unsup), C.byref(n)) == P.PL_EUNSUPPORTED
+    toomany = P.make_config((64, 64), [], append_cap=4)
+    assert P.lib.pl_workspace_bytes(C.byref(toomany), C.byref(n)) == P.PL_EINVAL
+    h = C.c_void_p()
+    assert P.lib.pl_ctx_create(C.byref(cfg), None, 0, C.byref(h)) == P.PL_EINVAL
+    assert P.lib.pl_ctx_create(C.byref(cfg), C.c_void_p(256), 16, C.byref(h)) == P.PL_ENOMEM
+
+
+def test_round_before_init_is_a_state_error():
+    import denoise_step_b200 as P
+    # a null context is rejected before any device work
+    assert P.lib.pl_stream_round(None, None, None, None, None, None, None, None, None) == P.PL_EINVAL
+    assert P.lib.pl_ring_push(None, None, None, None) == P.PL_EINVAL
