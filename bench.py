@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Throughput of the streaming pyramid denoising round (PersonaLive) on B200.
+
+One step = one whole round at 512x512 geometry: ring push of the new window,
+16 reference-attention layers in the SD-UNet layout (64x64/C320, 32x32/C640,
+16x16/C1280, 8x8/C1280, 8 heads) over [own ; bank x4] with the motion
+cross-attention after each, the pyramid DDIM step on 16x4x64x64 latents with
+the pop of the t=0 window, and the bank check of the 4 new motion embeddings.
+All inputs are seeded synthetic tensors of the pages' shapes (no weights or
+datasets exist here); per-round inputs (about 0.4 GB of hidden states) are
+larger than the 126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). N > 1 runs N independent replicas (one stream
+per GPU; the path has no exchange step), timed as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as S  # noqa: E402
+
+METRIC = "pyramid rounds/s & output frames/s; attn TFLOP/s as % of B200 FP16 peak"
+WORKLOAD = ("full round at 512x512 geometry: 16 reference-attention layers in SD-UNet layout "
+            "(64x64/C320 x5, 32x32/C640 x5, 16x16/C1280 x5, 8x8/C1280 x1; 8 heads), "
+            "KV = own + bank x4, motion x-attn 32x16-d per layer, DDIM on 16x4x64x64, bank check")
+SEED = S.SEEDS["full"]
+
+
+def attn_flops_layer(N: int, C: int, kv_entries: int = 5, frames: int = 16) -> float:
+    """Algorithmic attention-core FLOPs of one layer: 4 * Nq * Nkv * head_dim per (frame, head)."""
+    hd = C // S.HEADS
+    return 4.0 * frames * S.HEADS * N * (kv_entries * N) * hd
+
+
+def round_attn_flops() -> float:
+    return sum(attn_flops_layer(side * side, C) for _, side, C in S.LAYERS)
+
+
+def round_proj_flops() -> float:
+    """QKV + O projections and motion Q + O projections, 2*M*N*K each."""
+    tot = 0.0
+    for _, side, C in S.LAYERS:
+        M = 16 * side * side
+        tot += 2.0 * M * C * (3 * C) + 3 * (2.0 * M * C * C)
+    return tot
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 6650.0, "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("attn.cu", "attn.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "denoise_step_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic():
+    """DRAM bytes per launch of the timed attention kernel from the committed ncu summary,
+    or None when the kernel source changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "attn_level64_bank4_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_hash") != kernel_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------- workload
+
+class Workload:
+    """Seeded inputs of the full round, uploaded to the device once."""
+
+    def __init__(self, torch, device):
+        self.torch = torch
+        L = S.LAYERS
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        self.weights = []
+        for name, side, C in L:
+            w = S.layer_weights(SEED, name, C, np.float16)
+            self.weights.append({
+                "w_qkv": dev(np.concatenate([w["wq"], w["wk"], w["wv"]], 1)), "w_o": dev(w["wo"]),
+                "m_q": dev(w["mq"]), "m_kv": dev(np.concatenate([w["mk"], w["mv"]], 1)),
+                "m_o": dev(w["mo"])})
+        self.ref_feats = [dev(S.bank_features(SEED, n, 0, s * s, C)) for n, s, C in L]
+        self.anchors = [dev(S.bank_features(SEED, n, a, s * s, C)) for a in (1, 2, 3) for n, s, C in L]
+        self.ref_latent = dev(S.normal(SEED, "ref_latent", (4, 64, 64), 1.0, np.float32))
+        self.prefill_eps = dev(S.normal(SEED, "prefill_eps", (12, 4, 64, 64), 1.0, np.float32))
+        e0 = S.normal(SEED, "walk/e0", (512,), 1.0, np.float64)
+        self.ref_motion = dev(e0.astype(np.float32))
+        self.drive0 = dev(S.normal(SEED, "drive0", (512,), 1.0, np.float32))
+        # per-round inputs (host copies kept pinned for the end-to-end leg)
+        self.h_hidden = [S.layer_hidden(SEED, n, 1, 16, s * s, C) for n, s, C in L]
+        steps = S.normal(SEED, "walk/steps", (4, 512), 3.0)
+        self.h_motion = (e0[None] + np.cumsum(steps, 0)).astype(np.float32)
+        self.h_noise = S.normal(SEED, "noise", (4, 4, 64, 64), 1.0, np.float32)
+        self.h_eps = S.normal(SEED, "eps", (16, 4, 64, 64), 1.0, np.float32)
+        self.hidden = [dev(h) for h in self.h_hidden]
+        self.motion, self.noise, self.eps = dev(self.h_motion), dev(self.h_noise), dev(self.h_eps)
+        self.out = torch.empty((4, 4, 64, 64), dtype=torch.float32, device=device)
+        self.flags = torch.zeros(4, dtype=torch.uint8, device=device)
+        self.layer_out = [torch.empty((16, s * s, C), dtype=torch.float16, device=device)
+                          for _, s, C in L]
+
+
+def clocks_sampler(device_index: int, path: str):
+    q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    try:
+        f = open(path, "w")
+        return subprocess.Popen(["nvidia-smi", f"--id={device_index}", f"--query-gpu={q}",
+                                 "--format=csv,noheader,nounits", "-lms", "200"],
+                                stdout=f, stderr=subprocess.DEVNULL), f
+    except Exception:
+        return None, None
+
+
+def clocks_summary(path: str):
+    try:
+        rows = [r.split(",") for r in open(path).read().strip().splitlines() if r.strip()]
+    except Exception:
+        return None
+    sm, mx, reasons = [], 0.0, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for r in rows:
+        try:
+            sm.append(float(r[1]))
+            mx = max(mx, float(r[2]))
+        except (ValueError, IndexError):
+            continue
+        for n, v in zip(names, r[5:9]):
+            if v.strip().lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return None
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- CPU oracle arm
+
+def oracle_round_sample():
+    """Time the fp64 oracle on a bounded sample of one round and extrapolate to a round.
+
+    Sample: every layer, frame 0, R = 8 and R = 32 query rows (the per-frame K/V
+    projection of [own ; bank x4] is the fixed part, the per-row attention the
+    linear part), extrapolated to 16 frames x all rows; plus the full pile
+    DDIM step and bank check. Returns (seconds per round, sample description).
+    """
+    import oracle as O
+    rng_rows = (8, 32)
+    total = 0.0
+    tok = O.motion_tokens(S.normal(SEED, "walk/e0", (512,)))
+    for name, side, C in S.LAYERS:
+        N = side * side
+        w = S.layer_weights(SEED, name, C, np.float16)
+        h = S.normal(SEED, f"{name}/hidden/sample", (N, C), 1.0, np.float16)
+        bank = [S.bank_features(SEED, name, b, N, C) for b in range(4)]
+        ts = []
+        for R in rng_rows:
+            rows = np.arange(min(R, N))
+            t0 = time.perf_counter()
+            O.layer_forward_frame(h, w, bank, tok, S.HEADS, rows=rows)
+            ts.append(time.perf_counter() - t0)
+        r1, r2 = min(rng_rows[0], N), min(rng_rows[1], N)
+        per_row = max(ts[1] - ts[0], 0.0) / max(r2 - r1, 1)
+        fixed = max(ts[0] - r1 * per_row, 0.0)
+        total += 16 * (fixed + N * per_row)
+    ref = S.normal(SEED, "ref_latent", (4, 64, 64))
+    pe = S.normal(SEED, "prefill_eps", (12, 4, 64, 64))
+    st = O.PyramidStream(ref, pe, S.normal(SEED, "walk/e0", (512,)), S.normal(SEED, "drive0", (512,)))
+    noise = S.normal(SEED, "noise", (4, 4, 64, 64))
+    eps = S.normal(SEED, "eps", (16, 4, 64, 64))
+    mot = S.normal(SEED, "mot", (4, 512), 3.0)
+    t0 = time.perf_counter()
+    st.round(noise, mot, eps)
+    total += time.perf_counter() - t0
+    desc = ("per layer: frame 0 with 8 and 32 query rows (fixed K/V projection + per-row "
+            "attention), extrapolated linearly to 16 frames x all rows; full DDIM/pile/bank")
+    return total, desc
+
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max(int(i.get("num_threads", 1)) for i in info) if info else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        oracle_round_sample()
+    secs = []
+    desc = ""
+    for _ in range(args.steps):
+        s, desc = oracle_round_sample()
+        secs.append(s)
+    per_round = sum(secs) / len(secs)
+    value = 1.0 / per_round
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "rounds/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_round * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "frames_per_s": 4 * value},
+        "cpu_baseline": {"value": value, "unit": "rounds/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "rounds/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def time_attention_kernel(torch, P, wl, stream, reps=10):
+    """Average duration of the dominant kernel: the 64x64-level attention over [own ; bank x4]
+    (16 frames x 8 heads x 4096 queries x 20480 keys, head_dim 40), launched as in the round."""
+    N, C = 4096, 320
+    qkv = torch.randn((16, N, 3 * C), device="cuda", dtype=torch.float16,
+                      generator=torch.Generator(device="cuda").manual_seed(SEED))
+    bank = torch.randn((4, N, 2 * C), device="cuda", dtype=torch.float16,
+                       generator=torch.Generator(device="cuda").manual_seed(SEED + 1))
+    segs = [(qkv[:, :, C:2 * C], qkv[:, :, 2 * C:])] + [(bank[b, :, :C], bank[b, :, C:]) for b in range(4)]
+    out = torch.empty((16, N, C), device="cuda", dtype=torch.float16)
+    q = qkv[:, :, :C]
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            P.segment_attention(q, segs, 8, 40, out=out, stream=stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            P.segment_attention(q, segs, 8, 40, out=out, stream=stream)
+        e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps / 1e3
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import denoise_step_b200 as P
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    wl = Workload(torch, "cuda")
+    cfg = P.make_config((64, 64), [(s * s, C) for _, s, C in S.LAYERS])
+    st = P.Stream(cfg)
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    st.bank_init(wl.weights, wl.ref_feats, wl.anchors, wl.ref_motion, wl.drive0, wl.ref_latent,
+                 wl.prefill_eps, stream=stream)
+
+    def step():
+        st.round(wl.noise, wl.motion, wl.hidden, wl.eps, wl.out, wl.flags, wl.layer_out,
+                 stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            step()
+    stream.synchronize()
+    state = st.state(stream)
+    if state["bank_count"] != 4 or state["device_status"] != 0:
+        raise RuntimeError(f"unexpected state after warm-up: {state}")
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    clk_path = os.path.join(ROOT, "gpurun_out", f"bench_clocks_r{rank}.csv")
+    os.makedirs(os.path.dirname(clk_path), exist_ok=True)
+    proc, fh = clocks_sampler(local_rank, clk_path)
+    time.sleep(0.3)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+    barrier()
+    if proc is not None:
+        proc.terminate()
+        proc.wait()
+        fh.close()
+    elapsed = e0.elapsed_time(e1) / 1e3
+    if dist is not None:
+        t = torch.tensor([elapsed], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+    if st.device_status(stream) != 0:
+        raise RuntimeError("device status word set during the timed region")
+
+    # end to end through the public API: pinned host inputs in, x0 frames out, every step
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    h_hidden = [pin(h) for h in wl.h_hidden]
+    h_noise, h_motion, h_eps = pin(wl.h_noise), pin(wl.h_motion), pin(wl.h_eps)
+    h_out = torch.empty((4, 4, 64, 64), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h_hidden + [h_noise, h_motion, h_eps])
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        for d, h in zip(wl.hidden, h_hidden):
+            d.copy_(h, non_blocking=True)
+        wl.noise.copy_(h_noise, non_blocking=True)
+        wl.motion.copy_(h_motion, non_blocking=True)
+        wl.eps.copy_(h_eps, non_blocking=True)
+        step()
+        h_out.copy_(wl.out, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    with torch.cuda.stream(stream):
+        e2e_step()
+        stream.synchronize()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        f1.record(stream)
+    barrier()
+    e2e_elapsed = f0.elapsed_time(f1) / 1e3
+    if dist is not None:
+        t = torch.tensor([e2e_elapsed], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_elapsed = float(t.item())
+
+    # dominant kernel, timed alone on the stream it is launched on
+    attn_s = time_attention_kernel(torch, P, wl, stream)
+    attn_fl = attn_flops_layer(4096, 320)
+    tf_peak, hbm_peak, peak_kind = peaks()
+    achieved = attn_fl / attn_s / 1e12
+
+    launches_per_round = 1 + 7 * len(S.LAYERS) + 3 + 3
+    value = world * args.steps / elapsed
+    line = {
+        "metric": METRIC, "value": value, "unit": "rounds/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {
+            "workload": WORKLOAD, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "frames_per_s": 4 * value,
+            "round_attn_tflop": round_attn_flops() / 1e12,
+            "round_proj_tflop": round_proj_flops() / 1e12,
+            "round_tflops_effective": (round_attn_flops() + round_proj_flops()) * args.steps / elapsed / 1e12 / world,
+            "attn_tflops_level64": achieved,
+            "attn_frac_fp16_peak": {"measured": achieved / tf_peak, "spec_2250": achieved / 2250.0},
+            "l2": "per-step inputs (~0.4 GB hidden + bank K/V) exceed the 126 MB L2; no flush",
+        },
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
+                     "frac": achieved / tf_peak, "traffic": ncu_traffic(),
+                     "kernel": "attn_kernel<40> (64x64 level, KV own + bank x4)",
+                     "peak_kind": f"{peak_kind} bf16 burst (fp16 dense rate is the same)",
+                     "launch_ms": attn_s * 1e3},
+        "e2e": {"value": world * e2e_steps / e2e_elapsed, "unit": "rounds/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_round * args.steps,
+    }
+    clk = clocks_summary(clk_path)
+    if clk is not None:
+        line["clocks"] = clk
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, desc = oracle_round_sample()
+        line["cpu_baseline"] = {"value": 1.0 / secs, "unit": "rounds/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    st.close()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    return run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -316,15 +316,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 }
 
 template <int HD>
+int set_attr() {
+  return cudaFuncSetAttribute(attn_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(Cfg<HD>::SMEM)) == cudaSuccess ? 0 : 4;
+}
+
+template <int HD>
 int launch_hd(const AttnParams& p, cudaStream_t stream) {
   using C = Cfg<HD>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(attn_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(C::SMEM)) != cudaSuccess)
-      return 4;
-    attr_done = true;
-  }
   dim3 grid((p.n_q + 255) / 256, p.heads, p.frames);
   attn_kernel<HD><<<grid, kThreads, C::SMEM, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? 0 : 4;
@@ -385,7 +384,18 @@ int attn_make_params(AttnParams* p, const void* q, int64_t ldq, int64_t q_fstrid
   return 0;
 }
 
+int attn_init() {
+  static int done = 0;
+  if (!done) {
+    if (set_attr<40>() || set_attr<64>() || set_attr<80>() || set_attr<128>() || set_attr<160>())
+      return 4;
+    done = 1;
+  }
+  return 0;
+}
+
 int attn_launch(const AttnParams& p, int head_dim, cudaStream_t stream) {
+  if (attn_init()) return 4;
   switch (head_dim) {
     case 40: return launch_hd<40>(p, stream);
     case 64: return launch_hd<64>(p, stream);

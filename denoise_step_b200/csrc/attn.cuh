@@ -38,6 +38,8 @@ struct AttnSegHost {
 int attn_make_params(AttnParams* p, const void* q, int64_t ldq, int64_t q_fstride,
                      const AttnSegHost* segs, int n_segs, int frames, int n_q, int heads,
                      int head_dim, void* out, int64_t ldo, int64_t out_fstride);
+// Set kernel attributes once (call outside stream capture). 0 on success.
+int attn_init();
 int attn_launch(const AttnParams& p, int head_dim, cudaStream_t stream);
 
 }  // namespace pl

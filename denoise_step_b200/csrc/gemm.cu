@@ -225,14 +225,19 @@ int gemm_make_problem(GemmProblem* p, const void* a, int64_t lda, const void* b,
   return 0;
 }
 
-int gemm_launch(GemmParams* params, cudaStream_t stream, int max_ctas) {
-  static bool attr_done = false;
-  if (!attr_done) {
+int gemm_init() {
+  static int done = 0;
+  if (!done) {
     if (cudaFuncSetAttribute(gemm_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes)) != cudaSuccess)
       return 4;
-    attr_done = true;
+    done = 1;
   }
+  return 0;
+}
+
+int gemm_launch(GemmParams* params, cudaStream_t stream, int max_ctas) {
+  if (gemm_init()) return 4;
   int total = 0;
   for (int i = 0; i < params->n_problems; ++i) {
     GemmProblem& pr = params->prob[i];

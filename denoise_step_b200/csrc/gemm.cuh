@@ -36,6 +36,8 @@ struct GemmParams {
 // Host helpers (gemm.cu).
 int gemm_make_problem(GemmProblem* p, const void* a, int64_t lda, const void* b, int64_t ldb,
                       void* c, int64_t ldc, int M, int N, int K, const int32_t* pred);
+// Set kernel attributes once (call outside stream capture). 0 on success.
+int gemm_init();
 // Launch a grouped GEMM over params->prob[0..n_problems). Fills tile ranges.
 int gemm_launch(GemmParams* params, cudaStream_t stream, int max_ctas);
 

@@ -452,6 +452,12 @@ pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_
   ctx->ws_bytes = workspace_bytes;
   layout(*cfg, ctx);
   pl::ddim_coefficients(&ctx->coef);
+  // kernel attributes and the SM count are set up here, outside any stream capture
+  num_sms();
+  if (pl::gemm_init() || pl::attn_init()) {
+    delete ctx;
+    return PL_ECUDA;
+  }
   // zero the device state so pl_get_state is meaningful before bank_init
   if (cudaMemset(ctx->st, 0, sizeof(pl::DevState)) != cudaSuccess) {
     delete ctx;

@@ -1,0 +1,97 @@
+"""Run one kernel of the round on a chosen shape (for timing and ncu captures).
+
+    python -m denoise_step_b200.microbench attn --frames 16 --n 4096 --c 320 --bank 4 --reps 3
+    python -m denoise_step_b200.microbench gemm --m 65536 --n 960 --k 320 --reps 3
+    python -m denoise_step_b200.microbench ddim --h 64 --w 64 --streams 1 --reps 3
+
+Inputs are seeded torch tensors on the device; prints the mean CUDA-event time
+per launch and the algorithmic throughput.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import torch
+
+import denoise_step_b200 as P
+
+
+def _time(fn, reps, stream):
+    with torch.cuda.stream(stream):
+        fn()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps / 1e3
+
+
+def attn(a, stream):
+    g = torch.Generator(device="cuda").manual_seed(a.seed)
+    C, N, F, hd = a.c, a.n, a.frames, a.c // a.heads
+    qkv = torch.randn((F, N, 3 * C), device="cuda", dtype=torch.float16, generator=g)
+    bank = torch.randn((max(a.bank, 1), N, 2 * C), device="cuda", dtype=torch.float16, generator=g)
+    segs = [(qkv[:, :, C:2 * C], qkv[:, :, 2 * C:])]
+    segs += [(bank[b, :, :C], bank[b, :, C:]) for b in range(a.bank)]
+    out = torch.empty((F, N, C), device="cuda", dtype=torch.float16)
+    fn = lambda: P.segment_attention(qkv[:, :, :C], segs, a.heads, hd, out=out, stream=stream)
+    t = _time(fn, a.reps, stream)
+    flops = 4.0 * F * a.heads * N * (N * (1 + a.bank)) * hd
+    return {"kernel": f"attn hd{hd}", "s": t, "tflops": flops / t / 1e12}
+
+
+def gemm(a, stream):
+    g = torch.Generator(device="cuda").manual_seed(a.seed)
+    A = torch.randn((a.m, a.k), device="cuda", dtype=torch.float16, generator=g)
+    B = torch.randn((a.k, a.n), device="cuda", dtype=torch.float16, generator=g) / a.k ** 0.5
+    Cm = torch.empty((a.m, a.n), device="cuda", dtype=torch.float16)
+    t = _time(lambda: P.gemm(A, B, out=Cm, stream=stream), a.reps, stream)
+    return {"kernel": "gemm", "s": t, "tflops": 2.0 * a.m * a.n * a.k / t / 1e12,
+            "gbs": 2.0 * (a.m * a.k + a.k * a.n + a.m * a.n) / t / 1e9}
+
+
+def ddim(a, stream):
+    st = P.Stream(P.make_config((a.h, a.w), []))
+    fe = 4 * a.h * a.w
+    g = torch.Generator(device="cuda").manual_seed(a.seed)
+    mk = lambda *s: torch.randn(s, device="cuda", dtype=torch.float32, generator=g)
+    st.bank_init([], [], None, mk(512), mk(512), mk(4, a.h, a.w), mk(12, 4, a.h, a.w), stream=stream)
+    noise, mot, eps = mk(4, 4, a.h, a.w), mk(4, 512), mk(16, 4, a.h, a.w)
+    out = torch.empty((4, 4, a.h, a.w), device="cuda", dtype=torch.float32)
+
+    def fn():
+        st.ring_push(noise, mot, stream=stream)
+        st.ddim_step(eps, out, stream=stream)
+
+    t = _time(fn, a.reps, stream)
+    # algorithmic bytes of the step: read x and eps of 16 frames, write 12 x_prev + 4 x0 (fp32)
+    byts = 4.0 * fe * (16 + 16 + 16)
+    return {"kernel": "ring push + ddim", "s": t, "gbs_ddim_bytes": byts / t / 1e9}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("what", choices=["attn", "gemm", "ddim"])
+    ap.add_argument("--frames", type=int, default=16)
+    ap.add_argument("--n", type=int, default=4096)
+    ap.add_argument("--c", type=int, default=320)
+    ap.add_argument("--heads", type=int, default=8)
+    ap.add_argument("--bank", type=int, default=4)
+    ap.add_argument("--m", type=int, default=65536)
+    ap.add_argument("--k", type=int, default=320)
+    ap.add_argument("--h", type=int, default=64)
+    ap.add_argument("--w", type=int, default=64)
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--seed", type=int, default=1002)
+    a = ap.parse_args()
+    stream = torch.cuda.Stream()
+    r = {"attn": attn, "gemm": gemm, "ddim": ddim}[a.what](a, stream)
+    print(json.dumps(r))
+
+
+if __name__ == "__main__":
+    main()

@@ -38,6 +38,19 @@ def attn_errors(got, want):
     return float(d.max()), float(d.mean()), float(rel)
 
 
+def scaled_gates(want):
+    """Scale of the attention gates for an output of RMS r: max(1, r).
+
+    The absolute gates hold for outputs of unit scale or below (the reference
+    attention's outputs have RMS ~ 0.02-0.4). The layer output after the motion
+    cross-attention carries the motion embedding's magnitude, which a sigma = 3
+    random walk raises to ~8 within two rounds; there the same gates apply to
+    the output divided by its RMS.
+    """
+    r = float(np.sqrt(np.mean(np.square(np.asarray(want, np.float64)))))
+    return max(1.0, r)
+
+
 # tolerances of the floating-point paths
 ATTN_MAX_ABS = 1e-2
 ATTN_MEAN_ABS = 1e-3

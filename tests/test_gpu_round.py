@@ -1,0 +1,165 @@
+"""GPU parity of whole rounds (pl_stream_round) against the oracle's deque state machine."""
+import numpy as np
+import pytest
+
+import oracle as O
+import synthetic as S
+from _gpu_util import (ATTN_MAX_ABS, ATTN_MEAN_ABS, DDIM_ABS, attn_errors, dev, host,
+                       layer_weights_np, pack_weights, scaled_gates)
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def P():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import denoise_step_b200 as P
+    return P
+
+
+class Case:
+    """Seeded inputs of a stream: weights, bank features, prefill, per-round inputs."""
+
+    def __init__(self, seed, layers, H, W, walk_sigma, n_anchor=3):
+        self.seed, self.layers, self.H, self.W = seed, layers, H, W
+        self.w = [layer_weights_np(seed, name, C) for name, _, C in layers]
+        self.ref_feats = [S.bank_features(seed, name, 0, side * side, C) for name, side, C in layers]
+        self.anchors = [[S.bank_features(seed, name, a, side * side, C) for name, side, C in layers]
+                        for a in range(1, 1 + n_anchor)]
+        self.ref_latent = S.normal(seed, "ref_latent", (4, H, W), 1.0, np.float32)
+        self.prefill_eps = S.normal(seed, "prefill_eps", (12, 4, H, W), 1.0, np.float32)
+        self.ref_motion = S.normal(seed, "walk/e0", (512,), 1.0, np.float32)
+        self.walk_sigma = walk_sigma
+        self.e = self.ref_motion.astype(np.float64)
+        self.drive0 = None
+
+    def next_motion(self, r):
+        steps = S.normal(self.seed, f"walk/step{r}", (4, 512), self.walk_sigma)
+        out = np.empty((4, 512), np.float32)
+        for j in range(4):
+            self.e = self.e + steps[j]
+            out[j] = self.e.astype(np.float32)
+            self.e = out[j].astype(np.float64)
+        return out
+
+    def round_inputs(self, r):
+        H, W = self.H, self.W
+        hidden = [S.layer_hidden(self.seed, name, r, 16, side * side, C)
+                  for name, side, C in self.layers]
+        noise = S.normal(self.seed, f"noise{r}", (4, 4, H, W), 1.0, np.float32)
+        eps = S.normal(self.seed, f"eps{r}", (16, 4, H, W), 1.0, np.float32)
+        return hidden, noise, eps
+
+
+def _setup(P, case):
+    layers = [(side * side, C) for _, side, C in case.layers]
+    cfg = P.make_config((case.H, case.W), layers)
+    st = P.Stream(cfg)
+    pw = [pack_weights(w) for w in case.w]
+    drive0 = S.normal(case.seed, "drive0", (512,), 1.0, np.float32)
+    dev_anchor = [dev(a) for an in case.anchors for a in an]
+    st.bank_init(pw, [dev(f) for f in case.ref_feats], dev_anchor, dev(case.ref_motion),
+                 dev(drive0), dev(case.ref_latent), dev(case.prefill_eps))
+    orc = O.PyramidStream(case.ref_latent, case.prefill_eps, case.ref_motion, drive0,
+                          state_dtype=np.float32)
+    return st, orc, pw
+
+
+def _kv_bank(case, li, n_entries):
+    return [case.ref_feats[li]] + [case.anchors[a][li] for a in range(n_entries - 1)]
+
+
+@pytest.mark.parametrize("walk_sigma", [3.0, 0.5])
+def test_tiny_rounds_match_oracle(P, walk_sigma):
+    # 16 frames, one 8x8 level (C = 1280, head_dim 160), latents 16x4x8x8
+    case = Case(S.SEEDS["tiny"], [("m", 8, 1280)], 8, 8, walk_sigma)
+    st, orc, _ = _setup(P, case)
+    stream = torch.cuda.Stream()
+    out = torch.empty((4, 4, 8, 8), dtype=torch.float32, device="cuda")
+    flags = torch.zeros(4, dtype=torch.uint8, device="cuda")
+    layer_out = [torch.empty((16, 64, 1280), dtype=torch.float16, device="cuda")]
+    for r in range(1, 6):
+        hidden, noise, eps = case.round_inputs(r)
+        mot = case.next_motion(r)
+        d_hidden = [dev(h) for h in hidden]
+        d_noise, d_mot, d_eps = dev(noise), dev(mot), dev(eps)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            st.round(d_noise, d_mot, d_hidden, d_eps, out, flags, layer_out, stream=stream)
+        stream.synchronize()
+        # oracle: append, layers on the batch, step + pop, bank check
+        n_kv = 1 + orc.appends
+        orc.append(noise, mot)
+        bm = orc.batch_motion()
+        got = host(layer_out[0])
+        for f in range(16):
+            want = O.layer_forward_frame(hidden[0][f], case.w[0], _kv_bank(case, 0, n_kv),
+                                         O.motion_tokens(bm[f]), 8)
+            mx, mean, rel = attn_errors(got[f], want)
+            g = scaled_gates(want)
+            assert mx <= ATTN_MAX_ABS * g and mean <= ATTN_MEAN_ABS * g, (r, f, mx, mean, rel, g)
+            assert rel < 2e-3, (r, f, rel)
+        want_x0 = orc.step_and_pop(eps)
+        _, _, want_flags = orc.check_bank(mot)
+        orc.rounds += 1
+        assert np.max(np.abs(host(out) - want_x0)) <= DDIM_ABS, r
+        assert list(host(flags)) == want_flags, r
+        s = st.state()
+        assert s["bank_count"] == len(orc.bank) and s["appends"] == orc.appends
+        assert [s["slot_t"][(s["head"] + k) & 3] for k in range(3)] == orc.batch_timesteps()
+        assert s["rounds"] == r and s["device_status"] == 0
+    if walk_sigma == 3.0:
+        assert orc.appends == 3
+    else:
+        assert orc.appends == 0
+    assert np.array_equal(st.motion_bank(), np.array(orc.bank, np.float32))
+    st.close()
+
+
+def test_full_geometry_rounds_spot_checked(P):
+    # 16 reference-attention layers in the SD-UNet layout, bank x4 after round 1,
+    # DDIM on 16x4x64x64, bank check; sampled rows of one layer per level
+    case = Case(S.SEEDS["full"], list(S.LAYERS), 64, 64, 3.0)
+    st, orc, _ = _setup(P, case)
+    stream = torch.cuda.Stream()
+    out = torch.empty((4, 4, 64, 64), dtype=torch.float32, device="cuda")
+    flags = torch.zeros(4, dtype=torch.uint8, device="cuda")
+    layer_out = [torch.empty((16, side * side, C), dtype=torch.float16, device="cuda")
+                 for _, side, C in case.layers]
+    check_layers = {0: "d00", 2: "d10", 4: "d20", 6: "m", 15: "u32"}
+    rows_all = S.uniform_int(case.seed, "rows", 24, 4096)
+    for r in range(1, 4):
+        hidden, noise, eps = case.round_inputs(r)
+        mot = case.next_motion(r)
+        d_hidden = [dev(h) for h in hidden]
+        d_noise, d_mot, d_eps = dev(noise), dev(mot), dev(eps)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            st.round(d_noise, d_mot, d_hidden, d_eps, out, flags, layer_out, stream=stream)
+        stream.synchronize()
+        n_kv = 1 + orc.appends
+        orc.append(noise, mot)
+        bm = orc.batch_motion()
+        for li in check_layers:
+            _, side, C = case.layers[li]
+            N = side * side
+            rows = np.unique(rows_all % N)
+            got = host(layer_out[li])
+            for f in (0, 9):
+                want = O.layer_forward_frame(hidden[li][f], case.w[li], _kv_bank(case, li, n_kv),
+                                             O.motion_tokens(bm[f]), 8, rows=rows)
+                mx, mean, rel = attn_errors(got[f][rows], want)
+                g = scaled_gates(want)
+                assert mx <= ATTN_MAX_ABS * g and mean <= ATTN_MEAN_ABS * g, (r, li, f, mx, mean, rel)
+                assert rel < 2e-3, (r, li, f, rel)
+        want_x0 = orc.step_and_pop(eps)
+        _, _, want_flags = orc.check_bank(mot)
+        assert np.max(np.abs(host(out) - want_x0)) <= DDIM_ABS, r
+        assert list(host(flags)) == want_flags
+        s = st.state()
+        assert s["appends"] == orc.appends and s["device_status"] == 0
+    assert orc.appends == 3
+    st.close()
