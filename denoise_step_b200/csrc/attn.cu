@@ -13,10 +13,25 @@
 // rescaled rarely; the final 1/l uses the same maximum as P, so the result is
 // the exact softmax up to rounding.
 //
-// Roles: warp 0 TMA producer (Q once, K/V tiles into a STAGES ring), warp 1
-// MMA issuer + TMEM owner, warps 4..7 softmax of query tile 0, warps 8..11
-// softmax of query tile 1. The MMA warp interleaves the two tiles so the
-// tensor pipe works on one tile while the other one's softmax runs.
+// Roles: warpgroup 0 = warp 0 TMA producer (Q once, K/V tiles into a STAGES
+// ring) + warp 1 MMA issuer and TMEM owner (warps 2, 3 idle); warpgroups 1
+// and 2 = softmax of query tiles 0 and 1. setmaxnreg moves registers from
+// warpgroup 0 (120 per thread) to the softmax warpgroups (184 per thread); the
+// launch is refused unless the kernel was compiled at 168 registers per
+// thread, the exact total that split needs. The MMA warp interleaves the two
+// tiles so the tensor pipe works on one tile while the other one's softmax
+// runs.
+//
+// The softmax is issue- and MUFU-bound (one exp2 per score at head_dim 40
+// against 160 tensor FLOPs), so its inner loop uses packed f32x2 FMAs,
+// 3-input max and one of two exp2 paths (EXPM): 0 = ex2.approx.f32 on the
+// MUFU pipe; 2 = MUFU for 3 of every 4 pairs and a degree-3 polynomial
+// on the FMA pipe for the 4th (Cody-Waite split 2^x = 2^n 2^f with n the
+// nearest integer, f in [-0.5, 0.5]; coefficients from exp2_poly.py).
+// Measured on B200 (level-64 kernel): ex2.approx.f32 issues 16 results per
+// clock per SM and ex2.approx.f16x2 only 8 instructions (the same 16 results),
+// so the f16x2 path was dropped; the polynomial split (EXPM 2) was 7% slower
+// than MUFU alone at this shape and is kept only as a compile-time option.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -29,28 +44,102 @@ namespace pl {
 
 namespace {
 
-template <int HD>
+template <int HD, int VAR = 0>
 struct Cfg {
-  static constexpr int BN = HD > 128 ? 64 : 128;         // keys per tile
+  // VAR 0: 128-key tiles, one S buffer per query tile (64 keys at head_dim 160);
+  // VAR 1: 64-key tiles, two S buffers per query tile where TMEM allows;
+  // VAR 2: 96-key tiles with two S buffers where they fit (head_dim <= 64),
+  //        else as VAR 0
+  static constexpr bool V2 = VAR == 2 && 4 * 96 + 2 * ((HD + 15) / 16 * 16) <= 512;
+  static constexpr int BN = V2 ? 96 : ((VAR == 1 || HD > 128) ? 64 : 128);  // keys per tile
   static constexpr int HDP = (HD + 15) / 16 * 16;         // PV MMA N, QK MMA K
   static constexpr int NBLK = (HD + 63) / 64;             // 64-column smem blocks
   static constexpr int KSTEPS = HDP / 16;
-  static constexpr int STAGES = NBLK == 1 ? 4 : 2;
+  // S buffers per query tile: 2 (S of the next KV tile is computed while the
+  // softmax works on this one) when 4 S buffers and 2 O accumulators fit in
+  // the 512 TMEM columns, else 1
+  static constexpr int SB = ((VAR == 1 || V2) && 4 * BN + 2 * HDP <= 512) ? 2 : 1;
   static constexpr uint32_t Q_BLK = 128 * 128;            // one 64-col block of a Q tile
   static constexpr uint32_t Q_BYTES = 2 * NBLK * Q_BLK;
   static constexpr uint32_t KV_BLK = BN * 128;
   static constexpr uint32_t K_BYTES = NBLK * KV_BLK;
   static constexpr uint32_t STAGE_BYTES = 2 * K_BYTES;    // K then V
-  static constexpr uint32_t O_COL = 2 * BN;               // TMEM column of O_0
-  static constexpr size_t SMEM = Q_BYTES + STAGES * STAGE_BYTES + 1024 + 256;
-  static_assert(2 * BN + 2 * HDP <= 512, "TMEM budget");
+  static constexpr int STAGES = (NBLK == 1 ? 8 : (NBLK == 2 ? 4 : 2)) * 64 / BN;
+  static_assert(BN % 32 == 0 && STAGES >= 2, "tile shape");
+  static constexpr uint32_t O_COL = 2 * SB * BN;          // TMEM column of O_0
+  static constexpr size_t SMEM = Q_BYTES + STAGES * STAGE_BYTES + 1024 + 512;
+  static_assert(2 * SB * BN + 2 * HDP <= 512, "TMEM budget");
+  static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 constexpr int kThreads = 384;
+constexpr int kRegsLaunch = 168;      // 384 x 168 >= 128 x 120 + 256 x 184
+constexpr int kRegsProducer = 120;
+constexpr int kRegsSoftmax = 184;
 
-template <int HD>
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float ex2_f32(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// fp16x2 of (lo, hi), lo in the low half
+__device__ __forceinline__ uint32_t h2_from(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// 2^x for a pair on the FMA pipe: n = nearest integer (1.5 * 2^23 shifter),
+// f = x - n in [-0.5, 0.5], 2^f by a degree-3 polynomial, 2^n added into the
+// exponent field. x is clamped to >= -126 so 2^n stays a normal number.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  const uint64_t shift = f2_pack(12582912.f, 12582912.f);
+  const uint64_t xc = f2_pack(x0, x1);
+  const uint64_t y = f2_add(xc, shift);
+  const uint64_t n = f2_add(y, f2_pack(-12582912.f, -12582912.f));
+  float n0, n1;
+  f2_unpack(n, n0, n1);
+  const uint64_t f = f2_add(xc, f2_pack(-n0, -n1));
+  uint64_t pz = f2_fma(f, f2_pack(0.055088684f, 0.055088684f), f2_pack(0.242604047f, 0.242604047f));
+  pz = f2_fma(pz, f, f2_pack(0.693276227f, 0.693276227f));
+  pz = f2_fma(pz, f, f2_pack(0.999928951f, 0.999928951f));
+  float y0, y1, p0, p1;
+  f2_unpack(y, y0, y1);
+  f2_unpack(pz, p0, p1);
+  const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(y0) << 23);
+  const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(y1) << 23);
+  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+}
+
+template <int HD, int EXPM, int VAR>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams p) {
-  using C = Cfg<HD>;
+  using C = Cfg<HD, VAR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -60,10 +149,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + C::STAGES;
-  uint64_t* s_full = kv_empty + C::STAGES;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_full = p_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 2);
+  uint64_t* s_full = kv_empty + C::STAGES;   // [2 tiles][SB]
+  uint64_t* p_full = s_full + 2 * C::SB;     // [2 tiles][2]
+  uint64_t* o_full = p_full + 4;             // [2 tiles], one phase per PV
+  uint64_t* o_final = o_full + 2;            // [2 tiles], one phase: the tile's last PV done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -71,6 +161,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   const int q_row0 = blockIdx.x * 256;
   const int head = blockIdx.y;
   const int frame = blockIdx.z;
+
+  // the K/V boxes the host encoded must match this kernel's key tile, or the
+  // TMA writes would not fit the stage buffers: refuse to run
+  if (p.box_rows != C::BN) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && p.status)
+      atomicOr(p.status, DEV_BADARG);
+    return;
+  }
 
   int n_active = p.n_total;
   if (p.n_extra != nullptr) {
@@ -86,10 +184,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
+    for (int b = 0; b < 2 * C::SB; ++b) mbar_init(&s_full[b], 1);
+    for (int b = 0; b < 4; ++b) mbar_init(&p_full[b], 128);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
       mbar_init(&o_full[i], 1);
+      mbar_init(&o_final[i], 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -100,6 +199,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // TMEM column of S buffer b of query tile i, and of O_i
+  auto s_col = [](int i, int b) { return static_cast<uint32_t>((i * C::SB + b) * C::BN); };
+  auto o_col = [](int i) { return static_cast<uint32_t>(C::O_COL + i * C::HDP); };
+
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
+  }
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -139,26 +245,38 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_f16_f32(128, C::BN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_f16_f32(128, C::HDP, 0, 1);
-      const uint32_t q_base = smem_u32(sQ);
-      const uint32_t kv_base = smem_u32(sKV);
-      auto issue_qk = [&](int i, int stage) {
-        const uint32_t a0 = q_base + i * C::NBLK * C::Q_BLK;
-        const uint32_t b0 = kv_base + stage * C::STAGE_BYTES;
+      // Descriptor templates: the start-address field (bits 0-13) holds
+      // address >> 4, so adding (byte offset >> 4) moves a descriptor inside
+      // shared memory; all offsets below are compile-time except the stage.
+      const uint64_t dq = desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk = desc_sw128(smem_u32(sKV), 16, 1024);
+      const uint64_t dv = desc_sw128(smem_u32(sKV) + C::K_BYTES, C::KV_BLK, 1024);
+      auto issue_qk = [&](int i, int stage, int b) {
+        const uint64_t a0 = dq + ((i * C::NBLK * C::Q_BLK) >> 4);
+        const uint64_t b0 = dk + ((stage * C::STAGE_BYTES) >> 4);
+        const uint32_t d = tmem + s_col(i, b);
 #pragma unroll
         for (int k = 0; k < C::KSTEPS; ++k) {
-          const uint64_t ad = desc_sw128(a0 + (k >> 2) * C::Q_BLK + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = desc_sw128(b0 + (k >> 2) * C::KV_BLK + (k & 3) * 32, 16, 1024);
-          mma_ss(tmem + i * C::BN, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+          const uint32_t off = ((k >> 2) * C::Q_BLK + (k & 3) * 32) >> 4;
+          const uint32_t offk = ((k >> 2) * C::KV_BLK + (k & 3) * 32) >> 4;
+          mma_ss(d, a0 + off, b0 + offk, idesc_qk, k > 0 ? 1u : 0u);
         }
+        mma_commit(&s_full[i * C::SB + b]);
       };
-      auto issue_pv = [&](int i, int stage, bool acc) {
-        const uint32_t v0 = kv_base + stage * C::STAGE_BYTES + C::K_BYTES;
+      // O_i (+)= P_i V with P read from S buffer b (fp16, two keys per column)
+      auto issue_pv = [&](int i, int stage, int b, bool acc) {
+        const uint64_t v0 = dv + ((stage * C::STAGE_BYTES) >> 4);
+        const uint32_t d = tmem + o_col(i);
+        const uint32_t a = tmem + s_col(i, b);
 #pragma unroll
-        for (int k = 0; k < C::BN / 16; ++k) {
-          const uint64_t bd = desc_sw128(v0 + k * 2048, C::KV_BLK, 1024);
-          mma_ts(tmem + C::O_COL + i * C::HDP, tmem + i * C::BN + k * 8, bd, idesc_pv,
-                 (acc || k > 0) ? 1u : 0u);
-        }
+        for (int k = 0; k < C::BN / 16; ++k)
+          mma_ts(d, a + k * 8, v0 + ((k * 2048) >> 4), idesc_pv, (acc || k > 0) ? 1u : 0u);
+        mma_commit(&o_full[i]);
+      };
+      auto wait_p = [&](int i, int jt) {
+        const bool r = mbar_wait(&p_full[i * 2 + (jt & 1)], (jt >> 1) & 1, abort_flag);
+        tc_fence_after();
+        return r;
       };
       bool ok = mbar_wait(q_full, 0, abort_flag);
       tc_fence_after();
@@ -170,21 +288,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         for (int lt = 0; lt < nt; ++lt) {
           if (!(ok = mbar_wait(&kv_full[stage], phase, abort_flag))) break;
           tc_fence_after();
-          issue_qk(0, stage);
-          mma_commit(&s_full[0]);
-          if (jt > 0) {
-            if (!(ok = mbar_wait(&p_full[1], (jt - 1) & 1, abort_flag))) break;
-            tc_fence_after();
-            issue_pv(1, prev_stage, jt - 1 > 0);
-            mma_commit(&o_full[1]);
-            mma_commit(&kv_empty[prev_stage]);
+          if constexpr (C::SB == 2) {
+            // S(jt) of both tiles first, then the PVs of the previous tile: the
+            // softmax finds S(jt) ready when it finishes P(jt - 1)
+            issue_qk(0, stage, jt & 1);
+            issue_qk(1, stage, jt & 1);
+            if (jt > 0) {
+              if (!(ok = wait_p(0, jt - 1))) break;
+              issue_pv(0, prev_stage, (jt - 1) & 1, jt - 1 > 0);
+              if (!(ok = wait_p(1, jt - 1))) break;
+              issue_pv(1, prev_stage, (jt - 1) & 1, jt - 1 > 0);
+              mma_commit(&kv_empty[prev_stage]);
+            }
+          } else {
+            // one S buffer per tile: PV(jt - 1) must be issued before S(jt)
+            // overwrites the P it reads (the tensor pipe runs them in order)
+            issue_qk(0, stage, 0);
+            if (jt > 0) {
+              if (!(ok = wait_p(1, jt - 1))) break;
+              issue_pv(1, prev_stage, 0, jt - 1 > 0);
+              mma_commit(&kv_empty[prev_stage]);
+            }
+            issue_qk(1, stage, 0);
+            if (!(ok = wait_p(0, jt))) break;
+            issue_pv(0, stage, 0, jt > 0);
           }
-          issue_qk(1, stage);
-          mma_commit(&s_full[1]);
-          if (!(ok = mbar_wait(&p_full[0], jt & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_pv(0, stage, jt > 0);
-          mma_commit(&o_full[0]);
           prev_stage = stage;
           if (++stage == C::STAGES) {
             stage = 0;
@@ -193,22 +321,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           ++jt;
         }
       }
-      if (ok && jt > 0 && mbar_wait(&p_full[1], (jt - 1) & 1, abort_flag)) {
-        tc_fence_after();
-        issue_pv(1, prev_stage, jt - 1 > 0);
-        mma_commit(&o_full[1]);
-        mma_commit(&kv_empty[prev_stage]);
+      if (ok && jt > 0) {
+        if constexpr (C::SB == 2) {
+          if (wait_p(0, jt - 1)) {
+            issue_pv(0, prev_stage, (jt - 1) & 1, jt - 1 > 0);
+            mma_commit(&o_final[0]);
+            if (wait_p(1, jt - 1)) {
+              issue_pv(1, prev_stage, (jt - 1) & 1, jt - 1 > 0);
+              mma_commit(&o_final[1]);
+              mma_commit(&kv_empty[prev_stage]);
+            }
+          }
+        } else {
+          // tile 0's last PV was issued inside the loop
+          mma_commit(&o_final[0]);
+          if (wait_p(1, jt - 1)) {
+            issue_pv(1, prev_stage, 0, jt - 1 > 0);
+            mma_commit(&o_final[1]);
+            mma_commit(&kv_empty[prev_stage]);
+          }
+        }
       }
     }
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     const int i = (warp - 4) >> 2;          // query tile of this warpgroup
     const int q4 = warp & 3;                // TMEM lane quadrant
     const int row = 32 * q4 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(32 * q4) << 16;
-    const uint32_t s_addr = tmem + lane_off + i * C::BN;
-    const uint32_t o_addr = tmem + lane_off + C::O_COL + i * C::HDP;
+    const uint32_t o_addr = tmem + lane_off + o_col(i);
     const float sl2 = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     int jt = 0;
@@ -217,33 +360,43 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       const int len = p.seg[sg].len;
       const int nt = (len + C::BN - 1) / C::BN;
       for (int lt = 0; lt < nt; ++lt) {
-        if (!(ok = mbar_wait(&s_full[i], jt & 1, abort_flag))) break;
+        const int b = C::SB == 2 ? (jt & 1) : 0;
+        const uint32_t use = C::SB == 2 ? static_cast<uint32_t>(jt >> 1) : static_cast<uint32_t>(jt);
+        if (!(ok = mbar_wait(&s_full[i * C::SB + b], use & 1, abort_flag))) break;
         tc_fence_after();
+        const uint32_t s_addr = tmem + lane_off + s_col(i, b);
         float s[C::BN];
 #pragma unroll
         for (int c = 0; c < C::BN; c += 32) tmem_ld32(s_addr + c, reinterpret_cast<uint32_t*>(s + c));
         tmem_wait_ld();
         const int valid = len - lt * C::BN;
-        float mx = -INFINITY;
         if (valid < C::BN) {
 #pragma unroll
-          for (int c = 0; c < C::BN; ++c) {
-            s[c] = c < valid ? s[c] : -INFINITY;
-            mx = fmaxf(mx, s[c]);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < C::BN; ++c) mx = fmaxf(mx, s[c]);
+          for (int c = 0; c < C::BN; ++c) s[c] = c < valid ? s[c] : -INFINITY;
         }
-        const float m_tile = mx * sl2;
+        // row max as 8 independent max3 chains (short dependency depth)
+        float mx[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx[a] = s[a];
+#pragma unroll
+        for (int c = 8; c + 16 <= C::BN; c += 16) {
+#pragma unroll
+          for (int a = 0; a < 8; ++a) mx[a] = max3f(mx[a], s[c + a], s[c + 8 + a]);
+        }
+        if constexpr (((C::BN - 8) % 16) != 0) {
+#pragma unroll
+          for (int a = 0; a < 8; ++a) mx[a] = fmaxf(mx[a], s[C::BN - 8 + a]);
+        }
+        const float m_tile = fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], fmaxf(mx[5], fmaxf(mx[6], mx[7])))) * sl2;
         const bool need = m_tile > m_run + 8.0f;
         float alpha = 1.0f;
         if (need) {
-          alpha = exp2f(m_run - m_tile);
+          alpha = ex2_f32(m_run - m_tile);
           m_run = m_tile;
         }
         l_run *= alpha;
         if (__any_sync(0xffffffffu, need && jt > 0)) {
+          // rescale O_i once PV(jt - 1) has landed in it
           if (!(ok = mbar_wait(&o_full[i], (jt - 1) & 1, abort_flag))) break;
           tc_fence_after();
 #pragma unroll
@@ -257,27 +410,46 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           }
           tmem_wait_st();
         }
+        const uint64_t sc2 = f2_pack(sl2, sl2);
+        const uint64_t nm2 = f2_pack(-m_run, -m_run);
         float sum = 0.f;
 #pragma unroll
         for (int c = 0; c < C::BN; c += 32) {
           uint32_t pk[16];
+          {
+            uint64_t accs[4] = {0, 0, 0, 0};
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = exp2f(fmaf(s[c + 2 * e], sl2, -m_run));
-            const float p1 = exp2f(fmaf(s[c + 2 * e + 1], sl2, -m_run));
-            sum += p0 + p1;
-            pk[e] = pack_half2(p0, p1);
+            for (int e = 0; e < 16; ++e) {
+              const uint64_t x = f2_fma(f2_pack(s[c + 2 * e], s[c + 2 * e + 1]), sc2, nm2);
+              uint64_t pp;
+              if (EXPM == 2 && (e & 3) == 3) {
+                pp = exp2_poly2(x);
+              } else {
+                float x0, x1;
+                f2_unpack(x, x0, x1);
+                pp = f2_pack(ex2_f32(x0), ex2_f32(x1));
+              }
+              accs[e & 3] = f2_add(accs[e & 3], pp);
+              float p0, p1;
+              f2_unpack(pp, p0, p1);
+              pk[e] = h2_from(p0, p1);
+            }
+            float a0, a1;
+            f2_unpack(f2_add(f2_add(accs[0], accs[1]), f2_add(accs[2], accs[3])), a0, a1);
+            sum += a0 + a1;
           }
           tmem_st16(s_addr + c / 2, pk);
         }
         tmem_wait_st();
         l_run += sum;
         tc_fence_before();
-        mbar_arrive(&p_full[i]);
+        mbar_arrive(&p_full[i * 2 + (jt & 1)]);
         ++jt;
       }
     }
-    if (ok && jt > 0 && mbar_wait(&o_full[i], (jt - 1) & 1, abort_flag)) {
+    // o_final has a single phase, so this wait cannot be satisfied by an
+    // earlier PV (with two S buffers the last two PVs can both be in flight)
+    if (ok && jt > 0 && mbar_wait(&o_final[i], 0, abort_flag)) {
       tc_fence_after();
       const float inv = 1.0f / l_run;
       const int grow = q_row0 + 128 * i + row;
@@ -315,17 +487,41 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   if (threadIdx.x == 0 && *abort_flag && p.status) atomicOr(p.status, DEV_TIMEOUT);
 }
 
+// Tile schedule per head dimension (measured on B200, level-64 shape): 96-key
+// tiles with two S buffers per query tile where TMEM holds them (head_dim <=
+// 64), 128-key tiles with one S buffer otherwise (64 keys at head_dim 160).
+template <int HD>
+constexpr int kVar = (HD <= 64) ? 2 : 0;
+constexpr int kExpMode = 0;   // exp2 on the MUFU pipe only
+
+int block_n(int head_dim) {
+  switch (head_dim) {
+    case 40: return Cfg<40, kVar<40>>::BN;
+    case 64: return Cfg<64, kVar<64>>::BN;
+    case 80: return Cfg<80, kVar<80>>::BN;
+    case 128: return Cfg<128, kVar<128>>::BN;
+    case 160: return Cfg<160, kVar<160>>::BN;
+    default: return 0;
+  }
+}
+
 template <int HD>
 int set_attr() {
-  return cudaFuncSetAttribute(attn_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(Cfg<HD>::SMEM)) == cudaSuccess ? 0 : 4;
+  constexpr int V = kVar<HD>;
+  // the setmaxnreg split needs exactly kRegsLaunch registers per thread at launch
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, attn_kernel<HD, kExpMode, V>) != cudaSuccess) return 4;
+  if (fa.numRegs != kRegsLaunch) return 4;
+  return cudaFuncSetAttribute(attn_kernel<HD, kExpMode, V>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(Cfg<HD, V>::SMEM)) == cudaSuccess ? 0 : 4;
 }
 
 template <int HD>
 int launch_hd(const AttnParams& p, cudaStream_t stream) {
-  using C = Cfg<HD>;
+  constexpr int V = kVar<HD>;
   dim3 grid((p.n_q + 255) / 256, p.heads, p.frames);
-  attn_kernel<HD><<<grid, kThreads, C::SMEM, stream>>>(p);
+  attn_kernel<HD, kExpMode, V><<<grid, kThreads, Cfg<HD, V>::SMEM, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? 0 : 4;
 }
 
@@ -350,7 +546,9 @@ int attn_make_params(AttnParams* p, const void* q, int64_t ldq, int64_t q_fstrid
     const uint32_t box[4] = {64, 1, static_cast<uint32_t>(box_rows_q), 1};
     if (encode_f16_tmap(&p->q, q, 4, dims, strides, box) != 0) return 2;
   }
-  const uint32_t bn = head_dim > 128 ? 64 : 128;
+  const int bn_i = block_n(head_dim);
+  if (bn_i == 0) return 7;
+  const uint32_t bn = static_cast<uint32_t>(bn_i);
   for (int s = 0; s < n_segs; ++s) {
     const AttnSegHost& h = segs[s];
     if (h.len < 1 || h.len > (1ll << 30) || h.ld % 8 || h.frame_stride % 8 || h.frame_stride < 0)
@@ -380,6 +578,7 @@ int attn_make_params(AttnParams* p, const void* q, int64_t ldq, int64_t q_fstrid
   p->heads = heads;
   p->frames = frames;
   p->scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
+  p->box_rows = bn_i;
   p->status = nullptr;
   return 0;
 }

@@ -25,6 +25,7 @@ struct AttnParams {
   int64_t ldo, out_fstride;
   int n_q, heads, frames;
   float scale_log2;            // log2(e) / sqrt(head_dim)
+  int box_rows;                // K/V tensor-map box rows; must equal the kernel's key tile
   uint32_t* status;
 };
 

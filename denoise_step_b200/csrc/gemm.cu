@@ -107,6 +107,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(kGemmBM, kGemmBN, 0, 1);
+      // descriptor templates for stage 0 (start-address field = address >> 4)
+      const uint64_t da = desc_sw128(smem_u32(smem), 16, 1024);
+      const uint64_t db = desc_sw128(smem_u32(smem) + kABytes, kBBlockBytes, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int acc_i = 0;
@@ -123,14 +126,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) break;
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + stage * kStageBytes);
-          const uint32_t b0 = a0 + kABytes;
+          const uint64_t ad = da + ((stage * kStageBytes) >> 4);
+          const uint64_t bd = db + ((stage * kStageBytes) >> 4);
 #pragma unroll
-          for (int k = 0; k < kGemmBK / 16; ++k) {
-            const uint64_t ad = desc_sw128(a0 + 32 * k, 16, 1024);
-            const uint64_t bd = desc_sw128(b0 + 2048 * k, kBBlockBytes, 1024);
-            mma_ss(d, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
-          }
+          for (int k = 0; k < kGemmBK / 16; ++k)
+            mma_ss(d, ad + ((32 * k) >> 4), bd + ((2048 * k) >> 4), idesc, (kb > 0 || k > 0) ? 1u : 0u);
           mma_commit(&empty[stage]);
           if (++stage == kStages) {
             stage = 0;

@@ -77,6 +77,7 @@ def test_tiny_rounds_match_oracle(P, walk_sigma):
     # 16 frames, one 8x8 level (C = 1280, head_dim 160), latents 16x4x8x8
     case = Case(S.SEEDS["tiny"], [("m", 8, 1280)], 8, 8, walk_sigma)
     st, orc, _ = _setup(P, case)
+    saw_keep = False        # a check that found the bank close enough (no append, room left)
     stream = torch.cuda.Stream()
     out = torch.empty((4, 4, 8, 8), dtype=torch.float32, device="cuda")
     flags = torch.zeros(4, dtype=torch.uint8, device="cuda")
@@ -103,7 +104,9 @@ def test_tiny_rounds_match_oracle(P, walk_sigma):
             assert mx <= ATTN_MAX_ABS * g and mean <= ATTN_MEAN_ABS * g, (r, f, mx, mean, rel, g)
             assert rel < 2e-3, (r, f, rel)
         want_x0 = orc.step_and_pop(eps)
-        _, _, want_flags = orc.check_bank(mot)
+        appends_before = orc.appends
+        _, mind2, want_flags = orc.check_bank(mot)
+        saw_keep |= any(f == 0 and d <= 289.0 for f, d in zip(want_flags, mind2)) and appends_before < 3
         orc.rounds += 1
         assert np.max(np.abs(host(out) - want_x0)) <= DDIM_ABS, r
         assert list(host(flags)) == want_flags, r
@@ -112,9 +115,9 @@ def test_tiny_rounds_match_oracle(P, walk_sigma):
         assert [s["slot_t"][(s["head"] + k) & 3] for k in range(3)] == orc.batch_timesteps()
         assert s["rounds"] == r and s["device_status"] == 0
     if walk_sigma == 3.0:
-        assert orc.appends == 3
+        assert orc.appends == 3          # step norm ~68 >> 17: the cap is reached in round 1
     else:
-        assert orc.appends == 0
+        assert saw_keep                  # step norm ~11: some checks stay below the threshold
     assert np.array_equal(st.motion_bank(), np.array(orc.bank, np.float32))
     st.close()
 
