@@ -1,6 +1,7 @@
 """Build libpl.so (all CUDA sources, sm_100a) in-tree with nvcc.
 
-Usage: python -m denoise_step_b200.build [--verbose]
+Usage: python denoise_step_b200/build.py [--verbose]
+(run as a file: importing the package loads the library this script builds)
 """
 from __future__ import annotations
 
