@@ -1,7 +1,7 @@
 """denoise_step_b200: the streaming pyramid denoising round on B200 (sm_100a).
 
 A thin ctypes binding over the C ABI in include/pl.h (libpl.so, built in-tree
-by `python -m denoise_step_b200.build`). Every step of the round runs in the
+by `python denoise_step_b200/build.py`). Every step of the round runs in the
 library's CUDA kernels; this module only marshals arguments (torch tensors
 supply device memory and streams). There is no CPU fallback: importing the
 package without the built library raises.
@@ -25,7 +25,7 @@ class PLError(RuntimeError):
 
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m denoise_step_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python denoise_step_b200/build.py`")
 lib = C.CDLL(LIB_PATH)
 
 vp, i32, i64, f32, sz = C.c_void_p, C.c_int, C.c_int64, C.c_float, C.c_size_t
@@ -66,6 +66,7 @@ _SIGS = {
                                    vp, i64, i64, vp]),
     "pl_ref_attention_workspace_bytes": (i32, [i32, i32, i32, i32, C.POINTER(sz)]),
     "pl_ref_attention": (i32, [vp, vp, vp, C.POINTER(vp), i32, i32, i32, i32, i32, vp, vp, sz, vp]),
+    "pl_ref_attention_noalloc": (i32, [vp, vp, vp, C.POINTER(vp), i32, i32, i32, i32, i32, vp, vp]),
     "pl_motion_xattn_workspace_bytes": (i32, [i32, i32, i32, C.POINTER(sz)]),
     "pl_motion_xattn": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),
     "pl_motion_bank_check": (i32, [vp, vp, vp, i32, i32, vp, i32, f32, i32, vp, vp, vp, vp]),
@@ -172,6 +173,20 @@ def ref_attention(hidden, w_qkv, w_o, bank_feats, heads, out=None, workspace=Non
     check(lib.pl_ref_attention(_ptr(_contig(hidden, "hidden")), _ptr(w_qkv), _ptr(w_o), arr, nb, F,
                                N, Cc, heads, _ptr(out), _ptr(workspace), workspace.numel(),
                                _stream(stream)), "pl_ref_attention")
+    return out
+
+
+def ref_attention_noalloc(hidden, w_qkv, w_o, bank_feats, heads, out=None, stream=None):
+    """ref_attention with the library's built-in scratch (no workspace argument)."""
+    import torch
+    F, N, Cc = hidden.shape
+    nb = len(bank_feats)
+    if out is None:
+        out = torch.empty_like(hidden)
+    arr = _ptr_array(bank_feats) if nb else None
+    check(lib.pl_ref_attention_noalloc(_ptr(_contig(hidden, "hidden")), _ptr(w_qkv), _ptr(w_o),
+                                       arr, nb, F, N, Cc, heads, _ptr(out), _stream(stream)),
+          "pl_ref_attention_noalloc")
     return out
 
 

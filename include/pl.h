@@ -110,6 +110,36 @@ pl_status pl_ref_attention(const void* hidden, const void* w_qkv, const void* w_
                            int c, int heads, void* out, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/* Scratch size behind pl_ref_attention_noalloc: 32 MiB per device. */
+#define PL_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* pl_ref_attention without a workspace argument (no counterpart in the
+ * pages: an interface convenience of this library).
+ *
+ * For callers that cannot allocate device memory: code embedded in a host
+ * application that owns every device allocation, a real-time thread that must
+ * not block in cudaMalloc/cudaFree (both may synchronise the device), or a
+ * plugin with no allocator of its own. They still pass hidden, the weights,
+ * the bank features and out, exactly as for pl_ref_attention; the
+ * intermediate Q/K/V, bank K/V and pre-projection output go to a file-scope
+ * device array of PL_NOALLOC_SCRATCH_BYTES instead of a caller workspace.
+ *
+ * - Problems whose pl_ref_attention_workspace_bytes exceeds
+ *   PL_NOALLOC_SCRATCH_BYTES are rejected with PL_ENOMEM before any device
+ *   work (e.g. the 16-frame 8x8/C1280 layer with one bank entry needs about
+ *   11 MB and fits; a 64x64/C320 layer does not).
+ * - The call allocates nothing. Its first call on a device looks up the
+ *   array's device address (cudaGetSymbolAddress) and caches it, so make that
+ *   first call outside any stream capture. Every device that has made a call
+ *   keeps the array until the process exits.
+ * - All calls share one array per device and it keeps the last call's
+ *   contents; nothing in it has to start at zero. Calls whose execution can
+ *   overlap on the GPU (other streams, other threads) race on the array:
+ *   order them on one stream or synchronise between them. */
+pl_status pl_ref_attention_noalloc(const void* hidden, const void* w_qkv, const void* w_o,
+                                   const void* const* bank_feats, int n_bank, int frames,
+                                   int n, int c, int heads, void* out, void* stream);
+
 /* Bytes of device workspace pl_motion_xattn needs. */
 pl_status pl_motion_xattn_workspace_bytes(int frames, int n, int c, size_t* bytes);
 
