@@ -64,6 +64,8 @@ _SIGS = {
     "pl_gemm_f16": (i32, [vp, i64, vp, i64, vp, i64, i32, i32, i32, vp]),
     "pl_segment_attention": (i32, [vp, i64, i64, C.POINTER(KVSegment), i32, i32, i32, i32, i32,
                                    vp, i64, i64, vp]),
+    "pl_pr_sink_attention": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, C.POINTER(vp),
+                                   C.POINTER(vp), i32, i32, i32, i32, vp, vp, vp, vp]),
     "pl_ref_attention_workspace_bytes": (i32, [i32, i32, i32, i32, C.POINTER(sz)]),
     "pl_ref_attention": (i32, [vp, vp, vp, C.POINTER(vp), i32, i32, i32, i32, i32, vp, vp, sz, vp]),
     "pl_ref_attention_noalloc": (i32, [vp, vp, vp, C.POINTER(vp), i32, i32, i32, i32, i32, vp, vp]),
@@ -156,6 +158,26 @@ def segment_attention(q, segments, heads, head_dim, out=None, stream=None):
                                    heads, head_dim, _ptr(out), out.stride(1), out.stride(0),
                                    _stream(stream)), "pl_segment_attention")
     return out
+
+
+def pr_sink_attention(q, own, sink, pool, pose_store, pose_query, rolling, heads, head_dim,
+                      out=None, retrieved=None, retrieved_d2=None, stream=None):
+    """PR-Sink block attention: own/sink (k, v) [n, ld]; pool (k, v) [n_pool, n, ld];
+    rolling: list of (k, v) [n, ld]; pose_store [n_pool, d] fp32, pose_query [d] fp32."""
+    import torch
+    n = q.shape[0]
+    if out is None:
+        out = torch.empty_like(q)
+    if retrieved is None:
+        retrieved = torch.zeros(1, dtype=torch.int32, device=q.device)
+    kr = _ptr_array([k for k, _ in rolling]) if rolling else None
+    vr = _ptr_array([v for _, v in rolling]) if rolling else None
+    check(lib.pl_pr_sink_attention(_ptr(q), _ptr(own[0]), _ptr(own[1]), _ptr(sink[0]), _ptr(sink[1]),
+                                   _ptr(pool[0]), _ptr(pool[1]), pool[0].shape[0], _ptr(pose_store),
+                                   _ptr(pose_query), pose_store.shape[1], kr, vr, len(rolling), n,
+                                   heads, head_dim, _ptr(out), _ptr(retrieved), _ptr(retrieved_d2),
+                                   _stream(stream)), "pl_pr_sink_attention")
+    return out, retrieved
 
 
 def ref_attention(hidden, w_qkv, w_o, bank_feats, heads, out=None, workspace=None, stream=None):

@@ -219,7 +219,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       uint32_t phase = 0;
       for (int sg = 0; sg < n_active && !*abort_flag; ++sg) {
         const AttnSeg& seg = p.seg[sg];
-        const int fr = seg.per_frame ? frame : 0;
+        int fr = seg.per_frame ? frame : 0;
+        if (seg.block_sel != nullptr) {
+          fr = *((volatile const int32_t*)seg.block_sel);
+          if (fr < 0 || fr >= seg.n_blocks) {   // out of range: attend block 0, flag it
+            if (p.status && blockIdx.x == 0 && blockIdx.y == 0) atomicOr(p.status, DEV_BADARG);
+            fr = 0;
+          }
+        }
         const int nt = (seg.len + C::BN - 1) / C::BN;
         for (int lt = 0; lt < nt; ++lt) {
           if (!mbar_wait(&kv_empty[stage], phase ^ 1, abort_flag)) break;
@@ -555,11 +562,13 @@ int attn_make_params(AttnParams* p, const void* q, int64_t ldq, int64_t q_fstrid
       return 1;
     if (h.ld < static_cast<int64_t>(heads) * head_dim) return 1;
     if ((reinterpret_cast<uintptr_t>(h.k) | reinterpret_cast<uintptr_t>(h.v)) & 15) return 1;
-    const bool per_frame = h.frame_stride != 0 && frames > 1;
-    const int64_t fs = per_frame ? h.frame_stride : h.len * h.ld;
+    const bool stacked = h.block_sel != nullptr;
+    if (stacked && (h.n_blocks < 1 || h.frame_stride <= 0)) return 1;
+    const bool per_frame = !stacked && h.frame_stride != 0 && frames > 1;
+    const int64_t fs = (per_frame || stacked) ? h.frame_stride : h.len * h.ld;
+    const uint64_t n4 = stacked ? static_cast<uint64_t>(h.n_blocks) : (per_frame ? frames : 1);
     const uint64_t dims[4] = {static_cast<uint64_t>(head_dim), static_cast<uint64_t>(heads),
-                              static_cast<uint64_t>(h.len),
-                              static_cast<uint64_t>(per_frame ? frames : 1)};
+                              static_cast<uint64_t>(h.len), n4};
     const uint64_t strides[3] = {static_cast<uint64_t>(head_dim) * 2,
                                  static_cast<uint64_t>(h.ld) * 2, static_cast<uint64_t>(fs) * 2};
     const uint32_t box[4] = {64, 1, bn, 1};
@@ -567,6 +576,8 @@ int attn_make_params(AttnParams* p, const void* q, int64_t ldq, int64_t q_fstrid
     if (encode_f16_tmap(&p->seg[s].v, h.v, 4, dims, strides, box) != 0) return 2;
     p->seg[s].len = static_cast<int>(h.len);
     p->seg[s].per_frame = per_frame ? 1 : 0;
+    p->seg[s].block_sel = h.block_sel;
+    p->seg[s].n_blocks = static_cast<int>(n4);
   }
   p->n_fixed = n_segs;
   p->n_total = n_segs;

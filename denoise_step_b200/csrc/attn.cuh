@@ -13,6 +13,9 @@ struct AttnSeg {
   CUtensorMap v;
   int len;
   int per_frame;   // 1: frame f reads its own rows, 0: shared by all frames
+  const int32_t* block_sel;  // when non-null: every frame reads block *block_sel
+                             // of a stacked segment (a retrieved cache block)
+  int n_blocks;              // blocks in a stacked segment
 };
 
 struct AttnParams {
@@ -33,6 +36,10 @@ struct AttnSegHost {
   const void* k;
   const void* v;
   int64_t len, ld, frame_stride;
+  // optional: `n_blocks` blocks stacked at `frame_stride`, the one attended
+  // chosen on the device by *block_sel (0 <= *block_sel < n_blocks)
+  int64_t n_blocks = 0;
+  const int32_t* block_sel = nullptr;
 };
 
 // Build params (tensor maps) on the host. Returns 0 on success.

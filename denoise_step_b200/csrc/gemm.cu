@@ -156,14 +156,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
       tc_fence_after();
       const int row = tc.m0 + row_in_tile;
       const uint32_t taddr = tmem + buf * kAccStride + (static_cast<uint32_t>(32 * q) << 16);
-      __half* crow = pr.c + static_cast<int64_t>(row) * pr.ldc;
+      __half* crow = static_cast<__half*>(pr.c) + static_cast<int64_t>(row) * pr.ldc;
+      float* frow = static_cast<float*>(pr.c) + static_cast<int64_t>(row) * pr.ldc;
 #pragma unroll 1
       for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
         uint32_t r[16];
         tmem_ld16(taddr + c0, r);
         tmem_wait_ld();
         const int col = tc.n0 + c0;
-        if (row < pr.M && col < pr.N) {
+        if (row < pr.M && col < pr.N && pr.out_f32) {
+          float4* dst = reinterpret_cast<float4*>(frow + col);
+#pragma unroll
+          for (int q4i = 0; q4i < 4; ++q4i)
+            dst[q4i] = make_float4(__uint_as_float(r[4 * q4i]), __uint_as_float(r[4 * q4i + 1]),
+                                   __uint_as_float(r[4 * q4i + 2]), __uint_as_float(r[4 * q4i + 3]));
+        } else if (row < pr.M && col < pr.N) {
           uint4 v0, v1;
           v0.x = pack_half2(__uint_as_float(r[0]), __uint_as_float(r[1]));
           v0.y = pack_half2(__uint_as_float(r[2]), __uint_as_float(r[3]));
@@ -196,9 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
 }  // namespace
 
 int gemm_make_problem(GemmProblem* p, const void* a, int64_t lda, const void* b, int64_t ldb,
-                      void* c, int64_t ldc, int M, int N, int K, const int32_t* pred) {
+                      void* c, int64_t ldc, int M, int N, int K, const int32_t* pred,
+                      bool out_f32) {
   if (M <= 0 || N <= 0 || K <= 0) return 1;
-  if (N % 16 || K % 8 || lda % 8 || ldb % 8 || ldc % 8) return 1;
+  if (N % 16 || K % 8 || lda % 8 || ldb % 8 || ldc % 8) return 1;   // 16-byte rows
   if (lda < K || ldb < N || ldc < N) return 1;
   if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b) |
        reinterpret_cast<uintptr_t>(c)) & 15)
@@ -215,8 +223,9 @@ int gemm_make_problem(GemmProblem* p, const void* a, int64_t lda, const void* b,
     const uint32_t box[2] = {64, 64};
     if (encode_f16_tmap(&p->b, b, 2, dims, strides, box) != 0) return 2;
   }
-  p->c = static_cast<__half*>(c);
+  p->c = c;
   p->ldc = ldc;
+  p->out_f32 = out_f32 ? 1 : 0;
   p->M = M;
   p->N = N;
   p->K = K;

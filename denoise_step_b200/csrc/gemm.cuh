@@ -18,8 +18,9 @@ constexpr int kGemmMaxProblems = 16;
 struct GemmProblem {
   CUtensorMap a;        // 2D {K, M}, box {64, 128}, 128B swizzle (K-major A)
   CUtensorMap b;        // 2D {N, K}, box {64, 64}, 128B swizzle (MN-major B)
-  __half* c;
-  int64_t ldc;
+  void* c;                    // fp16, or fp32 when out_f32
+  int64_t ldc;                // elements
+  int out_f32;
   int M, N, K;
   int tiles_n;
   int tile_begin, tile_end;   // linear tile range [begin, end)
@@ -35,7 +36,8 @@ struct GemmParams {
 
 // Host helpers (gemm.cu).
 int gemm_make_problem(GemmProblem* p, const void* a, int64_t lda, const void* b, int64_t ldb,
-                      void* c, int64_t ldc, int M, int N, int K, const int32_t* pred);
+                      void* c, int64_t ldc, int M, int N, int K, const int32_t* pred,
+                      bool out_f32 = false);
 // Set kernel attributes once (call outside stream capture). 0 on success.
 int gemm_init();
 // Launch a grouped GEMM over params->prob[0..n_problems). Fills tile ranges.

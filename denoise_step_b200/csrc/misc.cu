@@ -181,15 +181,15 @@ constexpr int kBankThreads = 256;
 __global__ void __launch_bounds__(kBankThreads) bank_check_kernel(
     float* bank, int32_t* count_p, int32_t* appends_p, int capacity, int dim,
     const float* __restrict__ queries, int nq, double thr2, int cap, int32_t* argmin,
-    double* min_d2, uint8_t* appended, DevState* st) {
+    double* min_d2, uint8_t* appended, DevState* st, int count_val) {
   __shared__ double w_best[kBankThreads / 32];
   __shared__ int w_idx[kBankThreads / 32];
   __shared__ int s_cnt, s_app, s_do_append;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int nwarps = kBankThreads / 32;
   if (threadIdx.x == 0) {
-    s_cnt = *count_p;
-    s_app = *appends_p;
+    s_cnt = count_p ? *count_p : count_val;
+    s_app = appends_p ? *appends_p : 0;
     if (st) {
       for (int a = 0; a < 4; ++a) st->anchor_fire[a] = 0;
     }
@@ -249,8 +249,8 @@ __global__ void __launch_bounds__(kBankThreads) bank_check_kernel(
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    *count_p = s_cnt;
-    *appends_p = s_app;
+    if (count_p) *count_p = s_cnt;
+    if (appends_p) *appends_p = s_app;
   }
 }
 
@@ -259,17 +259,15 @@ struct PeTable {
   float v[32][16];
 };
 
-// tokens[f][p][c] = fp16(motion[f][16 p + c] + PE[p][c]);
-// kv[f][p][n] = sum_c tokens[f][p][c] * m_kv[c][n] (fp32 accumulate), n < 2C.
+// tok[p][c] = motion[f][16 p + c] + PE[p][c] (fp32);
+// kv[f][p][n] = sum_c tok[p][c] * m_kv[c][n] (fp32), n < 2C.
 __global__ void motion_kv_kernel(const float* __restrict__ motion, const __half* __restrict__ m_kv,
-                                 int C, __half* tokens, __half* kv, PeTable pe) {
+                                 int C, float* kv, PeTable pe) {
   __shared__ float tok[32][16];
   const int f = blockIdx.y;
   for (int i = threadIdx.x; i < 512; i += blockDim.x) {
     const int p = i >> 4, c = i & 15;
-    const __half h = __float2half_rn(motion[f * 512 + i] + pe.v[p][c]);
-    tok[p][c] = __half2float(h);
-    if (blockIdx.x == 0) tokens[f * 512 + i] = h;
+    tok[p][c] = motion[f * 512 + i] + pe.v[p][c];
   }
   __syncthreads();
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
@@ -281,47 +279,41 @@ __global__ void motion_kv_kernel(const float* __restrict__ motion, const __half*
     float acc = 0.f;
 #pragma unroll
     for (int c = 0; c < 16; ++c) acc = fmaf(tok[p][c], w[c], acc);
-    kv[(static_cast<int64_t>(f) * 32 + p) * 2 * C + n] = __float2half_rn(acc);
+    kv[(static_cast<int64_t>(f) * 32 + p) * 2 * C + n] = acc;
   }
 }
 
 // One thread per (query row, head): 32 scores in registers, smem-resident
 // K/V of the frame and head (fp32), softmax in fp32.
 template <int HD>
-__global__ void __launch_bounds__(128) motion_attn_kernel(const __half* __restrict__ q, int64_t ldq,
-                                                          const __half* __restrict__ kv, int N,
+__global__ void __launch_bounds__(128) motion_attn_kernel(const float* __restrict__ q, int64_t ldq,
+                                                          const float* __restrict__ kv, int N,
                                                           int C, __half* __restrict__ out,
                                                           int64_t ldo, float scale) {
   __shared__ float sk[32][HD];
   __shared__ float sv[32][HD];
   const int f = blockIdx.z, h = blockIdx.y;
-  const __half* kvf = kv + static_cast<int64_t>(f) * 32 * 2 * C;
+  const float* kvf = kv + static_cast<int64_t>(f) * 32 * 2 * C;
   for (int i = threadIdx.x; i < 32 * HD; i += blockDim.x) {
     const int p = i / HD, d = i % HD;
-    sk[p][d] = __half2float(kvf[p * 2 * C + h * HD + d]);
-    sv[p][d] = __half2float(kvf[p * 2 * C + C + h * HD + d]);
+    sk[p][d] = kvf[p * 2 * C + h * HD + d];
+    sv[p][d] = kvf[p * 2 * C + C + h * HD + d];
   }
   __syncthreads();
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
-  const __half* qr = q + (static_cast<int64_t>(f) * N + n) * ldq + h * HD;
+  const float* qr = q + (static_cast<int64_t>(f) * N + n) * ldq + h * HD;
   float s[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) s[j] = 0.f;
-  for (int d0 = 0; d0 < HD; d0 += 8) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(qr + d0);
-    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-    float qv[8];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 t = __half22float2(h2[e]);
-      qv[2 * e] = t.x;
-      qv[2 * e + 1] = t.y;
-    }
+  for (int d0 = 0; d0 < HD; d0 += 4) {
+    const float4 qv = *reinterpret_cast<const float4*>(qr + d0);
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s[j] = fmaf(qv[e], sk[j][d0 + e], s[j]);
+      s[j] = fmaf(qv.x, sk[j][d0], s[j]);
+      s[j] = fmaf(qv.y, sk[j][d0 + 1], s[j]);
+      s[j] = fmaf(qv.z, sk[j][d0 + 2], s[j]);
+      s[j] = fmaf(qv.w, sk[j][d0 + 3], s[j]);
     }
   }
   float mx = -INFINITY;
@@ -402,12 +394,21 @@ cudaError_t launch_bank_check(float* bank, int32_t* count, int32_t* appends, int
                               int32_t* argmin, double* min_d2, uint8_t* appended,
                               DevState* st, cudaStream_t s) {
   bank_check_kernel<<<1, kBankThreads, 0, s>>>(bank, count, appends, capacity, dim, queries, nq,
-                                               thr2, cap, argmin, min_d2, appended, st);
+                                               thr2, cap, argmin, min_d2, appended, st, 0);
   return cudaGetLastError();
 }
 
-cudaError_t launch_motion_kv(const float* motion, const __half* m_kv, int F, int C,
-                             __half* tokens, __half* kv, cudaStream_t s) {
+cudaError_t launch_nearest(const float* store, int count, int dim, const float* query,
+                           int32_t* argmin, double* min_d2, cudaStream_t s) {
+  // a bank check with no append allowed: the nearest stored vector
+  bank_check_kernel<<<1, kBankThreads, 0, s>>>(const_cast<float*>(store), nullptr, nullptr, count,
+                                               dim, query, 1, 0.0, 0, argmin, min_d2, nullptr,
+                                               nullptr, count);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_motion_kv(const float* motion, const __half* m_kv, int F, int C, float* kv,
+                             cudaStream_t s) {
   PeTable pe;
   for (int p = 0; p < 32; ++p)
     for (int i = 0; i < 8; ++i) {
@@ -416,11 +417,11 @@ cudaError_t launch_motion_kv(const float* motion, const __half* m_kv, int F, int
       pe.v[p][2 * i + 1] = static_cast<float>(std::cos(ang));
     }
   dim3 grid((2 * C + 255) / 256, F);
-  motion_kv_kernel<<<grid, 256, 0, s>>>(motion, m_kv, C, tokens, kv, pe);
+  motion_kv_kernel<<<grid, 256, 0, s>>>(motion, m_kv, C, kv, pe);
   return cudaGetLastError();
 }
 
-cudaError_t launch_motion_attn(const __half* q, int64_t ldq, const __half* kv, int F, int N,
+cudaError_t launch_motion_attn(const float* q, int64_t ldq, const float* kv, int F, int N,
                                int C, int heads, __half* out, int64_t ldo, cudaStream_t s) {
   const int hd = C / heads;
   dim3 grid((N + 127) / 128, heads, F);

@@ -47,11 +47,15 @@ cudaError_t launch_bank_check(float* bank, int32_t* count, int32_t* appends, int
                               int dim, const float* queries, int nq, double thr2, int cap,
                               int32_t* argmin, double* min_d2, uint8_t* appended,
                               DevState* st, cudaStream_t s);
-// tokens (fp16 [F][32][16]) and motion K/V (fp16 [F][32][2C]) of every frame.
-cudaError_t launch_motion_kv(const float* motion, const __half* m_kv, int F, int C,
-                             __half* tokens, __half* kv, cudaStream_t s);
-// out[f*N + n][h*hd + d] = softmax_j(q . k_j / sqrt(hd)) v_j, 32 keys per frame.
-cudaError_t launch_motion_attn(const __half* q, int64_t ldq, const __half* kv, int F, int N,
+// argmin_j ||query - store_j||^2 over `count` stored vectors (fp64, lowest index on ties).
+cudaError_t launch_nearest(const float* store, int count, int dim, const float* query,
+                           int32_t* argmin, double* min_d2, cudaStream_t s);
+// Motion K/V (fp32 [F][32][2C]) of every frame from tokens = motion + PE (fp32).
+cudaError_t launch_motion_kv(const float* motion, const __half* m_kv, int F, int C, float* kv,
+                             cudaStream_t s);
+// out[f*N + n][h*hd + d] = softmax_j(q . k_j / sqrt(hd)) v_j, 32 keys per frame;
+// q fp32 (the Mq projection's fp32 accumulators), K/V fp32, out fp16.
+cudaError_t launch_motion_attn(const float* q, int64_t ldq, const float* kv, int F, int N,
                                int C, int heads, __half* out, int64_t ldo, cudaStream_t s);
 
 }  // namespace pl

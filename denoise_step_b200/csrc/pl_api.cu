@@ -59,13 +59,12 @@ struct pl_ctx {
   float* slot_motion;
   float* batch_motion;
   float* bank;
-  __half* tokens;
   __half* bank_kv[PL_MAX_LAYERS];
-  __half* motion_kv[PL_MAX_LAYERS];
+  float* motion_kv[PL_MAX_LAYERS];   // fp32 [16][32][2C]
   __half* qkv;
   __half* attn_o;
   __half* a1;
-  __half* qm;
+  float* qm;                          // fp32 motion queries (Mq accumulators)
   __half* om;
   __half* out_default;
   pl::DdimCoef coef;
@@ -98,22 +97,21 @@ size_t layout(const pl_config& c, pl_ctx* ctx) {
   uint8_t* sm = take(sizeof(float) * 16 * 512);
   uint8_t* bm = take(sizeof(float) * 16 * 512);
   uint8_t* bank = take(sizeof(float) * capacity * 512);
-  uint8_t* tok = take(sizeof(__half) * 16 * 32 * 16);
   int64_t max_nc = 0;
   for (int l = 0; l < c.n_layers; ++l) {
     const int64_t N = c.layer_tokens[l], C = c.layer_channels[l];
     uint8_t* bkv = take(sizeof(__half) * capacity * N * 2 * C);
-    uint8_t* mkv = take(sizeof(__half) * 16 * 32 * 2 * C);
+    uint8_t* mkv = take(sizeof(float) * 16 * 32 * 2 * C);
     if (ctx) {
       ctx->bank_kv[l] = reinterpret_cast<__half*>(bkv);
-      ctx->motion_kv[l] = reinterpret_cast<__half*>(mkv);
+      ctx->motion_kv[l] = reinterpret_cast<float*>(mkv);
     }
     if (16 * N * C > max_nc) max_nc = 16 * N * C;
   }
   uint8_t* qkv = take(sizeof(__half) * 3 * max_nc);
   uint8_t* ao = take(sizeof(__half) * max_nc);
   uint8_t* a1 = take(sizeof(__half) * max_nc);
-  uint8_t* qm = take(sizeof(__half) * max_nc);
+  uint8_t* qm = take(sizeof(float) * max_nc);
   uint8_t* om = take(sizeof(__half) * max_nc);
   uint8_t* od = take(sizeof(__half) * max_nc);
   if (ctx) {
@@ -122,11 +120,10 @@ size_t layout(const pl_config& c, pl_ctx* ctx) {
     ctx->slot_motion = reinterpret_cast<float*>(sm);
     ctx->batch_motion = reinterpret_cast<float*>(bm);
     ctx->bank = reinterpret_cast<float*>(bank);
-    ctx->tokens = reinterpret_cast<__half*>(tok);
     ctx->qkv = reinterpret_cast<__half*>(qkv);
     ctx->attn_o = reinterpret_cast<__half*>(ao);
     ctx->a1 = reinterpret_cast<__half*>(a1);
-    ctx->qm = reinterpret_cast<__half*>(qm);
+    ctx->qm = reinterpret_cast<float*>(qm);
     ctx->om = reinterpret_cast<__half*>(om);
     ctx->out_default = reinterpret_cast<__half*>(od);
   }
@@ -172,11 +169,13 @@ pl_status project_bank(pl_ctx* ctx, const void* const* feats, int entry, const i
 }
 
 pl_status single_gemm(const void* a, int64_t lda, const void* b, int64_t ldb, void* c,
-                      int64_t ldc, int M, int N, int K, uint32_t* status, cudaStream_t s) {
+                      int64_t ldc, int M, int N, int K, uint32_t* status, cudaStream_t s,
+                      bool out_f32 = false) {
   GemmParams gp;
   std::memset(&gp, 0, sizeof(gp));
   gp.status = status;
-  const int r = pl::gemm_make_problem(&gp.prob[0], a, lda, b, ldb, c, ldc, M, N, K, nullptr);
+  const int r =
+      pl::gemm_make_problem(&gp.prob[0], a, lda, b, ldb, c, ldc, M, N, K, nullptr, out_f32);
   if (r) return gemm_status(r);
   gp.n_problems = 1;
   return gemm_status(pl::gemm_launch(&gp, s, num_sms()));
@@ -205,7 +204,7 @@ pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
     const pl_layer_weights& w = ctx->w[l];
     __half* out = a.layer_out ? static_cast<__half*>(a.layer_out[l]) : ctx->out_default;
     r = from_cuda(pl::launch_motion_kv(ctx->batch_motion, static_cast<const __half*>(w.m_kv), 16,
-                                       C, ctx->tokens, ctx->motion_kv[l], s));
+                                       C, ctx->motion_kv[l], s));
     if (r) return r;
     r = single_gemm(a.hidden[l], C, w.w_qkv, 3 * C, ctx->qkv, 3 * C, static_cast<int>(M), 3 * C,
                     C, &ctx->st->status, s);
@@ -231,7 +230,7 @@ pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
                     &ctx->st->status, s);
     if (r) return r;
     r = single_gemm(ctx->a1, C, w.m_q, C, ctx->qm, C, static_cast<int>(M), C, C,
-                    &ctx->st->status, s);
+                    &ctx->st->status, s, /*out_f32=*/true);
     if (r) return r;
     r = from_cuda(pl::launch_motion_attn(ctx->qm, C, ctx->motion_kv[l], 16, N, C, H, ctx->om, C, s));
     if (r) return r;
@@ -312,6 +311,46 @@ pl_status pl_segment_attention(const void* q, int64_t ldq, int64_t q_frame_strid
   return lr == 0 ? PL_OK : lr == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
 }
 
+pl_status pl_pr_sink_attention(const void* q, const void* k_own, const void* v_own,
+                               const void* k_sink, const void* v_sink, const void* k_pool,
+                               const void* v_pool, int n_pool, const float* pose_store,
+                               const float* pose_query, int pose_dim,
+                               const void* const* k_roll, const void* const* v_roll,
+                               int n_roll, int n, int heads, int head_dim, void* out,
+                               int32_t* retrieved, double* retrieved_d2, void* stream) {
+  if (!q || !k_own || !v_own || !k_sink || !v_sink || !k_pool || !v_pool || !pose_store ||
+      !pose_query || !out || !retrieved)
+    return PL_EINVAL;
+  if (n_pool < 1 || n_pool > 65536 || pose_dim < 1 || pose_dim > 4096 || n < 1 || heads < 1)
+    return PL_EINVAL;
+  if (n_roll < 0 || n_roll > pl::kAttnMaxSegs - 3 || (n_roll > 0 && (!k_roll || !v_roll)))
+    return PL_EINVAL;
+  if (!head_dim_supported(head_dim)) return PL_EUNSUPPORTED;
+  const int64_t ld = static_cast<int64_t>(heads) * head_dim;
+  AttnSegHost segs[pl::kAttnMaxSegs];
+  int ns = 0;
+  segs[ns++] = {k_own, v_own, n, ld, 0};
+  segs[ns++] = {k_sink, v_sink, n, ld, 0};
+  AttnSegHost pool{k_pool, v_pool, n, ld, static_cast<int64_t>(n) * ld};
+  pool.n_blocks = n_pool;
+  pool.block_sel = retrieved;
+  segs[ns++] = pool;
+  for (int r = 0; r < n_roll; ++r) {
+    if (!k_roll[r] || !v_roll[r]) return PL_EINVAL;
+    segs[ns++] = {k_roll[r], v_roll[r], n, ld, 0};
+  }
+  AttnParams p;
+  const int mr = pl::attn_make_params(&p, q, ld, static_cast<int64_t>(n) * ld, segs, ns, 1, n,
+                                      heads, head_dim, out, ld, static_cast<int64_t>(n) * ld);
+  if (mr) return mr == 1 ? PL_EINVAL : PL_ECUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  pl_status r = from_cuda(pl::launch_nearest(pose_store, n_pool, pose_dim, pose_query, retrieved,
+                                             retrieved_d2, s));
+  if (r) return r;
+  const int lr = pl::attn_launch(p, head_dim, s);
+  return lr == 0 ? PL_OK : lr == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
+}
+
 pl_status pl_ref_attention_workspace_bytes(int frames, int n, int c, int n_bank, size_t* bytes) {
   if (!bytes || frames < 1 || n < 1 || c < 1 || n_bank < 0 || n_bank > PL_MAX_BANK)
     return PL_EINVAL;
@@ -375,8 +414,8 @@ pl_status pl_ref_attention(const void* hidden, const void* w_qkv, const void* w_
 pl_status pl_motion_xattn_workspace_bytes(int frames, int n, int c, size_t* bytes) {
   if (!bytes || frames < 1 || n < 1 || c < 1) return PL_EINVAL;
   const size_t fnc = static_cast<size_t>(frames) * n * c;
-  *bytes = align_up(2 * static_cast<size_t>(frames) * 512) +
-           align_up(2 * static_cast<size_t>(frames) * 32 * 2 * c) + 2 * align_up(2 * fnc);
+  *bytes = align_up(4 * static_cast<size_t>(frames) * 32 * 2 * c) + align_up(4 * fnc) +
+           align_up(2 * fnc);
   return PL_OK;
 }
 
@@ -393,17 +432,15 @@ pl_status pl_motion_xattn(const void* x, const float* motion, const void* m_q, c
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t fnc = static_cast<size_t>(frames) * n * c;
   uint8_t* w = static_cast<uint8_t*>(workspace);
-  __half* tok = reinterpret_cast<__half*>(w);
-  w += align_up(2 * static_cast<size_t>(frames) * 512);
-  __half* kv = reinterpret_cast<__half*>(w);
-  w += align_up(2 * static_cast<size_t>(frames) * 32 * 2 * c);
-  __half* qm = reinterpret_cast<__half*>(w);
-  w += align_up(2 * fnc);
+  float* kv = reinterpret_cast<float*>(w);
+  w += align_up(4 * static_cast<size_t>(frames) * 32 * 2 * c);
+  float* qm = reinterpret_cast<float*>(w);
+  w += align_up(4 * fnc);
   __half* om = reinterpret_cast<__half*>(w);
   pl_status r = from_cuda(pl::launch_motion_kv(motion, static_cast<const __half*>(m_kv), frames,
-                                               c, tok, kv, s));
+                                               c, kv, s));
   if (r) return r;
-  r = single_gemm(x, c, m_q, c, qm, c, frames * n, c, c, nullptr, s);
+  r = single_gemm(x, c, m_q, c, qm, c, frames * n, c, c, nullptr, s, /*out_f32=*/true);
   if (r) return r;
   r = from_cuda(pl::launch_motion_attn(qm, c, kv, frames, n, c, heads, om, c, s));
   if (r) return r;

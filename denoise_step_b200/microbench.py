@@ -2,7 +2,8 @@
 
     python -m denoise_step_b200.microbench attn --frames 16 --n 4096 --c 320 --bank 4 --reps 3
     python -m denoise_step_b200.microbench gemm --m 65536 --n 960 --k 320 --reps 3
-    python -m denoise_step_b200.microbench ddim --h 64 --w 64 --streams 1 --reps 3
+    python -m denoise_step_b200.microbench ddim --h 64 --w 64 --reps 3
+    python -m denoise_step_b200.microbench sink --n 4096 --c 5120 --heads 40 --pool 64 --reps 3
 
 Inputs are seeded torch tensors on the device; prints the mean CUDA-event time
 per launch and the algorithmic throughput.
@@ -44,6 +45,27 @@ def attn(a, stream):
     return {"kernel": f"attn hd{hd}", "s": t, "tflops": flops / t / 1e12}
 
 
+def sink(a, stream):
+    """PR-Sink block: 4096 tokens, 40 heads x 128, KV = own + sink + retrieved + 3 rolling."""
+    g = torch.Generator(device="cuda").manual_seed(a.seed)
+    n, heads, hd, n_pool = a.n, a.heads, a.c // a.heads, a.pool
+    Cc = heads * hd
+    mk = lambda *s: torch.randn(s, device="cuda", dtype=torch.float16, generator=g)
+    q = mk(n, Cc)
+    own, snk = (mk(n, Cc), mk(n, Cc)), (mk(n, Cc), mk(n, Cc))
+    pool = (mk(n_pool, n, Cc), mk(n_pool, n, Cc))
+    roll = [(mk(n, Cc), mk(n, Cc)) for _ in range(3)]
+    store = torch.randn((n_pool, 64), device="cuda", generator=g)
+    pq = torch.randn((64,), device="cuda", generator=g)
+    out = torch.empty_like(q)
+    ret = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fn = lambda: P.pr_sink_attention(q, own, snk, pool, store, pq, roll, heads, hd, out=out,
+                                     retrieved=ret, stream=stream)
+    t = _time(fn, a.reps, stream)
+    flops = 4.0 * n * (6 * n) * hd * heads
+    return {"kernel": f"pr-sink attn hd{hd} x{heads}", "s": t, "tflops": flops / t / 1e12}
+
+
 def gemm(a, stream):
     g = torch.Generator(device="cuda").manual_seed(a.seed)
     A = torch.randn((a.m, a.k), device="cuda", dtype=torch.float16, generator=g)
@@ -75,7 +97,8 @@ def ddim(a, stream):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["attn", "gemm", "ddim"])
+    ap.add_argument("what", choices=["attn", "gemm", "ddim", "sink"])
+    ap.add_argument("--pool", type=int, default=64)
     ap.add_argument("--frames", type=int, default=16)
     ap.add_argument("--n", type=int, default=4096)
     ap.add_argument("--c", type=int, default=320)
@@ -89,7 +112,7 @@ def main():
     ap.add_argument("--seed", type=int, default=1002)
     a = ap.parse_args()
     stream = torch.cuda.Stream()
-    r = {"attn": attn, "gemm": gemm, "ddim": ddim}[a.what](a, stream)
+    r = {"attn": attn, "gemm": gemm, "ddim": ddim, "sink": sink}[a.what](a, stream)
     print(json.dumps(r))
 
 

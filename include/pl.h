@@ -93,6 +93,28 @@ pl_status pl_segment_attention(const void* q, int64_t ldq, int64_t q_frame_strid
                                int heads, int head_dim, void* out, int64_t ldo,
                                int64_t out_frame_stride, void* stream);
 
+/* PR-Sink bounded attention of one block (LiveAnimate page, PR-Sink: a
+ * bounded KV cache of a static sink block, one dynamic block retrieved by
+ * pose and a rolling buffer of three slots; attention within the query block
+ * is full, as in block-causal generation):
+ *   j* = argmin_j ||pose_query - pose_store[j]||^2   (fp64, lowest j on ties)
+ *   out = softmax(q K_cat^T / sqrt(head_dim)) V_cat,
+ *   K_cat = [k_own ; k_sink ; k_pool[j*] ; k_roll[0..n_roll)] (V alike).
+ * The retrieval runs on the device and feeds the attention directly (no host
+ * round trip). q, every k / v, out: device fp16 [n][heads*head_dim];
+ * k_pool / v_pool: device fp16 [n_pool][n][heads*head_dim]; pose_store:
+ * device fp32 [n_pool][pose_dim]; pose_query: device fp32 [pose_dim];
+ * k_roll / v_roll: host arrays of n_roll (0..5) device pointers; retrieved:
+ * device int32 [1] (written: j*); retrieved_d2: device double [1] or NULL.
+ * head_dim in {40, 64, 80, 128, 160}; 1 <= n_pool <= 65536. */
+pl_status pl_pr_sink_attention(const void* q, const void* k_own, const void* v_own,
+                               const void* k_sink, const void* v_sink, const void* k_pool,
+                               const void* v_pool, int n_pool, const float* pose_store,
+                               const float* pose_query, int pose_dim,
+                               const void* const* k_roll, const void* const* v_roll,
+                               int n_roll, int n, int heads, int head_dim, void* out,
+                               int32_t* retrieved, double* retrieved_d2, void* stream);
+
 /* Bytes of device workspace pl_ref_attention needs. */
 pl_status pl_ref_attention_workspace_bytes(int frames, int n, int c, int n_bank,
                                            size_t* bytes);
@@ -147,8 +169,11 @@ pl_status pl_motion_xattn_workspace_bytes(int frames, int n, int c, size_t* byte
  * expression embedding becomes 32 tokens x 16 channels plus a sinusoidal
  * position code; cross_attention_dim 16; 8 heads):
  *   tok[f] = reshape(motion[f], 32, 16) + PE  (PE[p,2i] = sin(p/10000^(2i/16)),
- *            PE[p,2i+1] = cos(same)), rounded to fp16;
- *   out = softmax((x Mq)(tok Mk)^T / sqrt(c/heads)) (tok Mv) Mo.
+ *            PE[p,2i+1] = cos(same)), in fp32;
+ *   out = softmax((x Mq)(tok Mk)^T / sqrt(c/heads)) (tok Mv) Mo,
+ * with the tokens, tok Mk / tok Mv and x Mq kept in fp32 (the embedding's
+ * magnitude grows along a stream, and fp16 there would be amplified by the
+ * softmax); x and the attention output enter the projections as fp16.
  * x: device fp16 [frames][n][c]; motion: device fp32 [frames][512];
  * m_q, m_o: device fp16 [c][c]; m_kv: device fp16 [16][2c] = [Mk|Mv];
  * out: device fp16 [frames][n][c]. */

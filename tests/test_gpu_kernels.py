@@ -237,3 +237,43 @@ def test_pile_ddim_prefill_and_state(P, H, W):
             assert np.max(np.abs(host(ring[slot]) - orc.pile[k].x)) <= DDIM_ABS, (r, k)
     assert np.array_equal(st.motion_bank(), np.array(orc.bank, np.float32))
     st.close()
+
+
+# ------------------------------------------------------------------ PR-Sink bounded attention
+
+def test_pr_sink_attention_retrieves_and_attends(P):
+    # 40 heads x head_dim 128; KV = query block + static sink + pose-retrieved block
+    # (argmin over 64 stored 64-d pose descriptors) + 3 rolling blocks; ragged block length
+    seed, n, heads, hd, n_pool = S.SEEDS["sink"], 1000, 40, 128, 64
+    Cc = heads * hd
+    g = lambda name, shape, std=1.0: S.normal(seed, name, shape, std, np.float16)
+    q = g("q", (n, Cc))
+    own = (g("k_own", (n, Cc)), g("v_own", (n, Cc)))
+    sink = (g("k_sink", (n, Cc)), g("v_sink", (n, Cc)))
+    roll = [(g(f"k_roll{r}", (n, Cc)), g(f"v_roll{r}", (n, Cc))) for r in range(3)]
+    store = S.normal(seed, "poses", (n_pool, 64), 1.0, np.float32)
+    pq = S.normal(seed, "pose_q", (64,), 1.0, np.float32)
+    target = O.pose_retrieve(store, pq)
+    # only the retrieved block carries full seeded values; the others are scaled
+    # copies of a small base, so attending the wrong block changes the output
+    base_k, base_v = g("pool_base_k", (n, Cc), 0.5), g("pool_base_v", (n, Cc), 0.5)
+    pool_k = torch.empty((n_pool, n, Cc), dtype=torch.float16, device="cuda")
+    pool_v = torch.empty_like(pool_k)
+    for j in range(n_pool):
+        pool_k[j] = dev(base_k) * (1.0 + j / n_pool)
+        pool_v[j] = dev(base_v) * (1.0 - j / (2 * n_pool))
+    tk, tv = g("pool_target_k", (n, Cc)), g("pool_target_v", (n, Cc))
+    pool_k[target] = dev(tk)
+    pool_v[target] = dev(tv)
+    d2 = torch.zeros(1, dtype=torch.float64, device="cuda")
+    out, ret = P.pr_sink_attention(dev(q), (dev(own[0]), dev(own[1])), (dev(sink[0]), dev(sink[1])),
+                                   (pool_k, pool_v), dev(store), dev(pq),
+                                   [(dev(k), dev(v)) for k, v in roll], heads, hd, retrieved_d2=d2)
+    torch.cuda.synchronize()
+    assert int(ret.item()) == target
+    assert abs(float(d2.item()) - O.sq_dist(pq, store[target])) <= 1e-12 * O.sq_dist(pq, store[target])
+    rows = np.unique(np.concatenate([S.uniform_int(seed, "rows", 40, n), [0, n - 1]]))
+    want = O.segment_attention(q[rows], [own[0], sink[0], tk] + [k for k, _ in roll],
+                               [own[1], sink[1], tv] + [v for _, v in roll], heads)
+    mx, mean, rel = attn_errors(host(out)[rows], want)
+    assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (mx, mean, rel)
