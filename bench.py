@@ -266,6 +266,79 @@ def time_attention_kernel(torch, P, wl, stream, reps=10):
     return e0.elapsed_time(e1) / reps / 1e3
 
 
+def _event_time(torch, fn, reps, stream):
+    with torch.cuda.stream(stream):
+        fn()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps / 1e3
+
+
+def secondary_measurements(torch, P, stream, hbm_peak):
+    """The other workloads' kernels, timed live (CUDA events on their stream):
+    the PR-Sink block (4096 tokens x 40 heads x 128, KV own + sink + retrieved
+    of 64 + 3 rolling), the pile DDIM step on a scaled latent grid (1024 x 1024:
+    ring + epsilon 512 MB, past L2), and the nearest-vector search over a 1 GB
+    store. Inputs are seeded torch tensors (timing only)."""
+    g = torch.Generator(device="cuda").manual_seed(SEED)
+    out = {}
+    # PR-Sink
+    n, heads, hd = 4096, 40, 128
+    Cc = heads * hd
+    mk = lambda *sh: torch.randn(sh, device="cuda", dtype=torch.float16, generator=g)
+    q = mk(n, Cc)
+    own, snk = (mk(n, Cc), mk(n, Cc)), (mk(n, Cc), mk(n, Cc))
+    pool = (mk(64, n, Cc), mk(64, n, Cc))
+    roll = [(mk(n, Cc), mk(n, Cc)) for _ in range(3)]
+    store = torch.randn((64, 64), device="cuda", generator=g)
+    pq = torch.randn((64,), device="cuda", generator=g)
+    o = torch.empty_like(q)
+    ret = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t = _event_time(torch, lambda: P.pr_sink_attention(q, own, snk, pool, store, pq, roll, heads,
+                                                       hd, out=o, retrieved=ret, stream=stream),
+                    5, stream)
+    fl = 4.0 * n * 6 * n * hd * heads
+    out["pr_sink_block"] = {"ms": t * 1e3, "tflops": fl / t / 1e12}
+    del q, own, snk, pool, roll, o
+    # DDIM pile step on a scaled latent grid
+    H = W = 1024
+    fe = 4 * H * W
+    st = P.Stream(P.make_config((H, W), []))
+    mkf = lambda *sh: torch.randn(sh, device="cuda", generator=g)
+    st.bank_init([], [], None, mkf(512), mkf(512), mkf(4, H, W), mkf(12, 4, H, W), stream=stream)
+    noise, mot, eps = mkf(4, 4, H, W), mkf(4, 512), mkf(16, 4, H, W)
+    xo = torch.empty((4, 4, H, W), device="cuda")
+
+    def ddim_round():
+        st.ring_push(noise, mot, stream=stream)
+        st.ddim_step(eps, xo, stream=stream)
+
+    t = _event_time(torch, ddim_round, 10, stream)
+    byts = 4.0 * fe * (8 + 48)   # push: 4 frames in + out; step: x, eps of 16 frames in, 16 out
+    out["ddim_pile_1024x1024"] = {"ms": t * 1e3, "gbs": byts / t / 1e9,
+                                  "frac_hbm": byts / t / 1e9 / hbm_peak}
+    st.close()
+    del noise, eps, xo
+    # nearest vector over a large store
+    count, dim = 1 << 21, 128
+    store = torch.randn((count, dim), device="cuda", generator=g)
+    qv = torch.randn((dim,), device="cuda", generator=g)
+    am = torch.zeros(1, dtype=torch.int64, device="cuda")
+    md = torch.zeros(1, dtype=torch.float64, device="cuda")
+    t = _event_time(torch, lambda: P.nearest(store, qv, am, md, stream=stream), 10, stream)
+    byts = 4.0 * count * dim
+    out["nearest_2M_x128"] = {"ms": t * 1e3, "gbs": byts / t / 1e9,
+                              "frac_hbm": byts / t / 1e9 / hbm_peak}
+    del store
+    torch.cuda.synchronize()
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import denoise_step_b200 as P
@@ -391,6 +464,8 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_round * args.steps,
     }
+    if rank == 0 and not args.no_secondary:
+        line["config"]["secondary"] = secondary_measurements(torch, P, stream, hbm_peak)
     clk = clocks_summary(clk_path)
     if clk is not None:
         line["clocks"] = clk
@@ -414,6 +489,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -72,6 +72,8 @@ _SIGS = {
     "pl_motion_xattn_workspace_bytes": (i32, [i32, i32, i32, C.POINTER(sz)]),
     "pl_motion_xattn": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),
     "pl_motion_bank_check": (i32, [vp, vp, vp, i32, i32, vp, i32, f32, i32, vp, vp, vp, vp]),
+    "pl_nearest_workspace_bytes": (i32, [i64, C.POINTER(sz)]),
+    "pl_nearest": (i32, [vp, i64, i32, vp, vp, vp, vp, sz, vp]),
     "pl_workspace_bytes": (i32, [C.POINTER(Config), C.POINTER(sz)]),
     "pl_ctx_create": (i32, [C.POINTER(Config), vp, sz, C.POINTER(vp)]),
     "pl_ctx_destroy": (i32, [vp]),
@@ -237,6 +239,24 @@ def motion_bank_check(bank, count, appends, queries, threshold, cap, argmin=None
                                    _ptr(queries), nq, float(threshold), int(cap), _ptr(argmin),
                                    _ptr(min_d2), _ptr(appended), _stream(stream)),
           "pl_motion_bank_check")
+
+
+def nearest(store, query, argmin=None, min_d2=None, workspace=None, stream=None):
+    """argmin_j ||query - store_j||^2 over a large fp32 store [count, dim] (one read)."""
+    import torch
+    count, dim = store.shape
+    need = sz()
+    check(lib.pl_nearest_workspace_bytes(count, C.byref(need)), "pl_nearest_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need.value, dtype=torch.uint8, device=store.device)
+    if argmin is None:
+        argmin = torch.zeros(1, dtype=torch.int64, device=store.device)
+    if min_d2 is None:
+        min_d2 = torch.zeros(1, dtype=torch.float64, device=store.device)
+    check(lib.pl_nearest(_ptr(_contig(store, "store")), count, dim, _ptr(query), _ptr(argmin),
+                         _ptr(min_d2), _ptr(workspace), workspace.numel(), _stream(stream)),
+          "pl_nearest")
+    return argmin, min_d2
 
 
 # --------------------------------------------------------------------------- stream context

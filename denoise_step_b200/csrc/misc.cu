@@ -22,10 +22,12 @@ void ddim_coefficients(DdimCoef* out) {
     const int t = ts[k];
     const double at = abar[t];
     const double ap = t - 333 >= 0 ? abar[t - 333] : 1.0;
-    out->c[k][0] = std::sqrt(at);
+    out->c[k][0] = 1.0 / std::sqrt(at);
     out->c[k][1] = std::sqrt(1.0 - at);
     out->c[k][2] = std::sqrt(ap);
     out->c[k][3] = std::sqrt(1.0 - ap);
+    out->fwd[k][0] = std::sqrt(at);
+    out->fwd[k][1] = std::sqrt(1.0 - at);
   }
 }
 
@@ -50,8 +52,8 @@ __global__ void prefill_kernel(DevState* st, float* ring, float* slot_motion, fl
     const int64_t e = i - k * frame_elems;
     const int w = static_cast<int>(k / 4);  // window 0..2 -> t = 0, 333, 666
     const int ti = 3 - w;                   // table index of t
-    const double x = coef.c[ti][0] * static_cast<double>(ref_latent[e]) +
-                     coef.c[ti][1] * static_cast<double>(prefill_eps[i]);
+    const double x = coef.fwd[ti][0] * static_cast<double>(ref_latent[e]) +
+                     coef.fwd[ti][1] * static_cast<double>(prefill_eps[i]);
     ring[i] = static_cast<float>(x);        // slot w, frame k % 4
   }
   // motion: 13-point ramp ref -> drive0 with the last point dropped
@@ -117,43 +119,37 @@ __global__ void ring_push_kernel(DevState* st, float* ring, float* slot_motion,
 }
 
 // ------------------------------------------------------------------ DDIM
-// Batch frame f belongs to window w = f / 4 (oldest first), physical slot
-// (head + w) & 3. Arithmetic in fp64, one rounding to fp32 per output.
+// Batch frame f = blockIdx.y belongs to window w = f / 4 (oldest first), in
+// physical slot (head + w) & 3. Arithmetic in fp64 (x0 via the precomputed
+// 1/sqrt(abar_t)), one rounding to fp32 per output.
 __global__ void ddim_kernel(const DevState* __restrict__ st, float* ring,
                             const float* __restrict__ eps, float* __restrict__ out_x0,
                             int64_t frame_elems, DdimCoef coef) {
-  const int head = st->head;
-  int tix[4], slot[4];
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    slot[w] = (head + w) & 3;
-    tix[w] = t_index(st->slot_t[slot[w]]);
-  }
+  const int f = blockIdx.y;
+  const int w = f >> 2, j = f & 3;
+  const int slot = (st->head + w) & 3;
+  const int ti = t_index(st->slot_t[slot]);
+  if (ti < 0) return;
+  const double isa = coef.c[ti][0], sb = coef.c[ti][1];
+  const double pa = coef.c[ti][2], pb = coef.c[ti][3];
   const int64_t fe4 = frame_elems / 4;
-  const int64_t total = 16 * fe4;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int f = static_cast<int>(i / fe4);
-    const int64_t e = i - f * fe4;
-    const int w = f >> 2, j = f & 3;
-    const int ti = tix[w];
-    if (ti < 0) continue;
-    float4* xp = reinterpret_cast<float4*>(ring) + (static_cast<int64_t>(slot[w]) * 4 + j) * fe4 + e;
-    const float4 x = *xp;
-    const float4 ep = reinterpret_cast<const float4*>(eps)[i];
-    const double sa = coef.c[ti][0], sb = coef.c[ti][1];
-    const double x0x = (x.x - sb * ep.x) / sa, x0y = (x.y - sb * ep.y) / sa;
-    const double x0z = (x.z - sb * ep.z) / sa, x0w = (x.w - sb * ep.w) / sa;
+  float4* xf = reinterpret_cast<float4*>(ring) + (static_cast<int64_t>(slot) * 4 + j) * fe4;
+  const float4* ef = reinterpret_cast<const float4*>(eps) + static_cast<int64_t>(f) * fe4;
+  float4* of = reinterpret_cast<float4*>(out_x0) + static_cast<int64_t>(j) * fe4;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < fe4;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 x = xf[e];
+    const float4 ep = ef[e];
+    const double x0x = (x.x - sb * ep.x) * isa, x0y = (x.y - sb * ep.y) * isa;
+    const double x0z = (x.z - sb * ep.z) * isa, x0w = (x.w - sb * ep.w) * isa;
     if (ti == 3) {
-      reinterpret_cast<float4*>(out_x0)[j * fe4 + e] =
-          make_float4(static_cast<float>(x0x), static_cast<float>(x0y), static_cast<float>(x0z),
-                      static_cast<float>(x0w));
+      of[e] = make_float4(static_cast<float>(x0x), static_cast<float>(x0y),
+                          static_cast<float>(x0z), static_cast<float>(x0w));
     } else {
-      const double pa = coef.c[ti][2], pb = coef.c[ti][3];
-      *xp = make_float4(static_cast<float>(pa * x0x + pb * ep.x),
-                        static_cast<float>(pa * x0y + pb * ep.y),
-                        static_cast<float>(pa * x0z + pb * ep.z),
-                        static_cast<float>(pa * x0w + pb * ep.w));
+      xf[e] = make_float4(static_cast<float>(pa * x0x + pb * ep.x),
+                          static_cast<float>(pa * x0y + pb * ep.y),
+                          static_cast<float>(pa * x0z + pb * ep.z),
+                          static_cast<float>(pa * x0w + pb * ep.w));
     }
   }
 }
@@ -348,6 +344,120 @@ __global__ void __launch_bounds__(128) motion_attn_kernel(const float* __restric
   }
 }
 
+// ------------------------------------------------------------------ nearest (large stores)
+// Pass 1: every warp takes whole entries (lanes stride the dimension with
+// 16-byte loads); d2 in fp64; each CTA keeps its first minimum and writes it
+// to part_d2 / part_idx[blockIdx.x]. Pass 2: one CTA reduces the partials,
+// lowest index on equal distances. One read of the store in total.
+constexpr int kNearThreads = 256;
+
+__global__ void __launch_bounds__(kNearThreads) nearest_partial_kernel(
+    const float* __restrict__ store, int64_t count, int dim, const float* __restrict__ query,
+    double* part_d2, int64_t* part_idx) {
+  __shared__ double w_best[kNearThreads / 32];
+  __shared__ int64_t w_idx[kNearThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * (kNearThreads / 32) + warp;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (kNearThreads / 32);
+  double best = INFINITY;
+  int64_t bidx = INT64_MAX;
+  const bool vec = (dim % 4) == 0 && dim <= 128;
+  constexpr int U = 4;   // entries per warp iteration (more loads in flight)
+  for (int64_t j0 = gw * U; j0 < count; j0 += nw * U) {
+    double acc[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) acc[u] = 0.0;
+    if (vec) {
+      // dim <= 128: one 16-byte chunk per lane and entry
+      const int d = 4 * lane;
+      float4 a[U];
+      float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (d < dim) q = *reinterpret_cast<const float4*>(query + d);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        a[u] = q;   // entries past the end contribute nothing
+        if (d < dim && j0 + u < count)
+          a[u] = *reinterpret_cast<const float4*>(store + (j0 + u) * dim + d);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const double d0 = static_cast<double>(q.x) - a[u].x, d1 = static_cast<double>(q.y) - a[u].y;
+        const double d2 = static_cast<double>(q.z) - a[u].z, d3 = static_cast<double>(q.w) - a[u].w;
+        acc[u] = fma(d3, d3, fma(d2, d2, fma(d1, d1, d0 * d0)));
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (j0 + u >= count) continue;
+        const float* e = store + (j0 + u) * dim;
+        for (int d = lane; d < dim; d += 32) {
+          const double df = static_cast<double>(query[d]) - e[d];
+          acc[u] = fma(df, df, acc[u]);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (j0 + u < count && acc[u] < best) {   // entries of a warp increase
+        best = acc[u];
+        bidx = j0 + u;
+      }
+    }
+  }
+  if (lane == 0) {
+    w_best[warp] = best;
+    w_idx[warp] = bidx;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double b = INFINITY;
+    int64_t bi = INT64_MAX;
+    for (int w = 0; w < kNearThreads / 32; ++w)
+      if (w_best[w] < b || (w_best[w] == b && w_idx[w] < bi)) {
+        b = w_best[w];
+        bi = w_idx[w];
+      }
+    part_d2[blockIdx.x] = b;
+    part_idx[blockIdx.x] = bi;
+  }
+}
+
+__global__ void nearest_reduce_kernel(const double* part_d2, const int64_t* part_idx, int parts,
+                                      int64_t* argmin, double* min_d2) {
+  __shared__ double sb[256];
+  __shared__ int64_t si[256];
+  double b = INFINITY;
+  int64_t bi = INT64_MAX;
+  for (int k = threadIdx.x; k < parts; k += blockDim.x)
+    if (part_d2[k] < b || (part_d2[k] == b && part_idx[k] < bi)) {
+      b = part_d2[k];
+      bi = part_idx[k];
+    }
+  sb[threadIdx.x] = b;
+  si[threadIdx.x] = bi;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) {
+      const double ob = sb[threadIdx.x + o];
+      const int64_t oi = si[threadIdx.x + o];
+      if (ob < sb[threadIdx.x] || (ob == sb[threadIdx.x] && oi < si[threadIdx.x])) {
+        sb[threadIdx.x] = ob;
+        si[threadIdx.x] = oi;
+      }
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    *argmin = si[0] == INT64_MAX ? -1 : si[0];
+    if (min_d2) *min_d2 = sb[0];
+  }
+}
+
 int grid_for(int64_t work, int threads) {
   int64_t g = (work + threads - 1) / threads;
   const int64_t cap = 148 * 16;
@@ -379,8 +489,8 @@ cudaError_t launch_ring_push(DevState* st, float* ring, float* slot_motion, floa
 
 cudaError_t launch_ddim(DevState* st, float* ring, const float* eps, float* out_x0,
                         int64_t frame_elems, const DdimCoef& coef, cudaStream_t s) {
-  ddim_kernel<<<grid_for(4 * frame_elems, 256), 256, 0, s>>>(st, ring, eps, out_x0, frame_elems,
-                                                            coef);
+  dim3 grid(static_cast<unsigned>((grid_for(frame_elems / 4, 256) + 15) / 16), 16);
+  ddim_kernel<<<grid, 256, 0, s>>>(st, ring, eps, out_x0, frame_elems, coef);
   return cudaGetLastError();
 }
 
@@ -404,6 +514,21 @@ cudaError_t launch_nearest(const float* store, int count, int dim, const float* 
   bank_check_kernel<<<1, kBankThreads, 0, s>>>(const_cast<float*>(store), nullptr, nullptr, count,
                                                dim, query, 1, 0.0, 0, argmin, min_d2, nullptr,
                                                nullptr, count);
+  return cudaGetLastError();
+}
+
+int nearest_parts(int64_t count) {
+  int64_t g = (count + (kNearThreads / 32) * 4 - 1) / ((kNearThreads / 32) * 4);
+  if (g > 148 * 8) g = 148 * 8;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+cudaError_t launch_nearest_large(const float* store, int64_t count, int dim, const float* query,
+                                 double* part_d2, int64_t* part_idx, int parts, int64_t* argmin,
+                                 double* min_d2, cudaStream_t s) {
+  nearest_partial_kernel<<<parts, kNearThreads, 0, s>>>(store, count, dim, query, part_d2,
+                                                        part_idx);
+  nearest_reduce_kernel<<<1, 256, 0, s>>>(part_d2, part_idx, parts, argmin, min_d2);
   return cudaGetLastError();
 }
 

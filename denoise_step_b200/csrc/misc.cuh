@@ -23,10 +23,12 @@ struct DevState {
 };
 
 // Per-timestep DDIM coefficients for the 4 timesteps of the table, in table
-// order t = 999, 666, 333, 0: {sqrt(abar_t), sqrt(1-abar_t), sqrt(abar_prev),
-// sqrt(1-abar_prev)} with abar_prev = 1 below t = 0.
+// order t = 999, 666, 333, 0: c = {1/sqrt(abar_t), sqrt(1-abar_t),
+// sqrt(abar_prev), sqrt(1-abar_prev)} with abar_prev = 1 below t = 0, and
+// fwd = {sqrt(abar_t), sqrt(1-abar_t)} for forward noising (the prefill).
 struct DdimCoef {
   double c[4][4];
+  double fwd[4][2];
 };
 
 // Host: fill the coefficients from the SD scaled-linear schedule.
@@ -50,6 +52,12 @@ cudaError_t launch_bank_check(float* bank, int32_t* count, int32_t* appends, int
 // argmin_j ||query - store_j||^2 over `count` stored vectors (fp64, lowest index on ties).
 cudaError_t launch_nearest(const float* store, int count, int dim, const float* query,
                            int32_t* argmin, double* min_d2, cudaStream_t s);
+// Nearest stored vector over a large store in one read: per-CTA partial
+// minima (parts of them, in caller memory), then a one-CTA reduction.
+int nearest_parts(int64_t count);
+cudaError_t launch_nearest_large(const float* store, int64_t count, int dim, const float* query,
+                                 double* part_d2, int64_t* part_idx, int parts, int64_t* argmin,
+                                 double* min_d2, cudaStream_t s);
 // Motion K/V (fp32 [F][32][2C]) of every frame from tokens = motion + PE (fp32).
 cudaError_t launch_motion_kv(const float* motion, const __half* m_kv, int F, int C, float* kv,
                              cudaStream_t s);

@@ -462,6 +462,31 @@ pl_status pl_motion_bank_check(float* bank, int32_t* count, int32_t* appends, in
                                          static_cast<cudaStream_t>(stream)));
 }
 
+pl_status pl_nearest_workspace_bytes(int64_t count, size_t* bytes) {
+  if (!bytes || count < 1 || count >= (1ll << 40)) return PL_EINVAL;
+  const int parts = pl::nearest_parts(count);
+  *bytes = align_up(sizeof(double) * parts) + align_up(sizeof(int64_t) * parts);
+  return PL_OK;
+}
+
+pl_status pl_nearest(const float* store, int64_t count, int dim, const float* query,
+                     int64_t* argmin, double* min_d2, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  if (!store || !query || !argmin || !workspace) return PL_EINVAL;
+  if (dim < 1 || dim > 65536) return PL_EINVAL;
+  size_t need = 0;
+  const pl_status v = pl_nearest_workspace_bytes(count, &need);
+  if (v) return v;
+  if (workspace_bytes < need) return PL_ENOMEM;
+  if (dim % 4 == 0 && (!aligned16(store) || !aligned16(query))) return PL_EINVAL;
+  const int parts = pl::nearest_parts(count);
+  double* pd = static_cast<double*>(workspace);
+  int64_t* pi = reinterpret_cast<int64_t*>(static_cast<uint8_t*>(workspace) +
+                                           align_up(sizeof(double) * parts));
+  return from_cuda(pl::launch_nearest_large(store, count, dim, query, pd, pi, parts, argmin,
+                                            min_d2, static_cast<cudaStream_t>(stream)));
+}
+
 pl_status pl_workspace_bytes(const pl_config* cfg, size_t* bytes) {
   if (!bytes) return PL_EINVAL;
   const pl_status v = validate_config(cfg);

@@ -4,6 +4,7 @@
     python -m denoise_step_b200.microbench gemm --m 65536 --n 960 --k 320 --reps 3
     python -m denoise_step_b200.microbench ddim --h 64 --w 64 --reps 3
     python -m denoise_step_b200.microbench sink --n 4096 --c 5120 --heads 40 --pool 64 --reps 3
+    python -m denoise_step_b200.microbench nearest --count 1048576 --dim 128 --reps 10
 
 Inputs are seeded torch tensors on the device; prints the mean CUDA-event time
 per launch and the algorithmic throughput.
@@ -66,6 +67,20 @@ def sink(a, stream):
     return {"kernel": f"pr-sink attn hd{hd} x{heads}", "s": t, "tflops": flops / t / 1e12}
 
 
+def nearest(a, stream):
+    """argmin over a large fp32 store (one read): algorithmic bytes = count * dim * 4."""
+    g = torch.Generator(device="cuda").manual_seed(a.seed)
+    store = torch.randn((a.count, a.dim), device="cuda", generator=g)
+    q = torch.randn((a.dim,), device="cuda", generator=g)
+    am = torch.zeros(1, dtype=torch.int64, device="cuda")
+    md = torch.zeros(1, dtype=torch.float64, device="cuda")
+    need = P.sz()
+    P.check(P.lib.pl_nearest_workspace_bytes(a.count, P.C.byref(need)), "ws")
+    ws = torch.empty(need.value, dtype=torch.uint8, device="cuda")
+    t = _time(lambda: P.nearest(store, q, am, md, ws, stream=stream), a.reps, stream)
+    return {"kernel": "nearest", "s": t, "gbs": 4.0 * a.count * a.dim / t / 1e9}
+
+
 def gemm(a, stream):
     g = torch.Generator(device="cuda").manual_seed(a.seed)
     A = torch.randn((a.m, a.k), device="cuda", dtype=torch.float16, generator=g)
@@ -97,7 +112,9 @@ def ddim(a, stream):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["attn", "gemm", "ddim", "sink"])
+    ap.add_argument("what", choices=["attn", "gemm", "ddim", "sink", "nearest"])
+    ap.add_argument("--count", type=int, default=1 << 20)
+    ap.add_argument("--dim", type=int, default=128)
     ap.add_argument("--pool", type=int, default=64)
     ap.add_argument("--frames", type=int, default=16)
     ap.add_argument("--n", type=int, default=4096)
@@ -112,7 +129,7 @@ def main():
     ap.add_argument("--seed", type=int, default=1002)
     a = ap.parse_args()
     stream = torch.cuda.Stream()
-    r = {"attn": attn, "gemm": gemm, "ddim": ddim, "sink": sink}[a.what](a, stream)
+    r = {"attn": attn, "gemm": gemm, "ddim": ddim, "sink": sink, "nearest": nearest}[a.what](a, stream)
     print(json.dumps(r))
 
 

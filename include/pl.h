@@ -198,6 +198,21 @@ pl_status pl_motion_bank_check(float* bank, int32_t* count, int32_t* appends, in
                                int cap, int32_t* argmin, double* min_d2, uint8_t* appended,
                                void* stream);
 
+/* Bytes of device workspace pl_nearest needs for a store of `count` entries. */
+pl_status pl_nearest_workspace_bytes(int64_t count, size_t* bytes);
+
+/* Nearest stored vector for large stores (LiveAnimate page, PR-Sink's pose
+ * retrieval; the motion-bank distance of the PersonaLive write-up,
+ * "抗身份漂移的补丁", without appends): argmin_j ||query - store_j||^2 with
+ * fp64 distances, lowest j on equal distances, reading the store once over
+ * the whole GPU. store: device fp32 [count][dim] (16-byte aligned rows when
+ * dim % 4 == 0); query: device fp32 [dim]; argmin: device int64 [1];
+ * min_d2: device double [1] or NULL; workspace: device, >=
+ * pl_nearest_workspace_bytes(count). 1 <= count < 2^40, 1 <= dim <= 65536. */
+pl_status pl_nearest(const float* store, int64_t count, int dim, const float* query,
+                     int64_t* argmin, double* min_d2, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
 /* ------------------------------------------------------------------ *
  * Stream context: the device-resident pile and the reference bank
  * ------------------------------------------------------------------ */

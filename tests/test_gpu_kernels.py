@@ -277,3 +277,20 @@ def test_pr_sink_attention_retrieves_and_attends(P):
                                [own[1], sink[1], tv] + [v for _, v in roll], heads)
     mx, mean, rel = attn_errors(host(out)[rows], want)
     assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (mx, mean, rel)
+
+
+# ------------------------------------------------------------------ nearest vector over a large store
+
+@pytest.mark.parametrize("count,dim", [(200000, 64), (50001, 30)])
+def test_nearest_large_store_bit_exact(P, count, dim):
+    seed = S.SEEDS["sink"]
+    store = S.normal(seed, f"store{count}", (count, dim), 1.0, np.float32)
+    q = S.normal(seed, f"q{count}", (dim,), 1.0, np.float32)
+    d2 = np.sum((store.astype(np.float64) - q.astype(np.float64)) ** 2, axis=1)
+    j = int(np.argmin(d2))
+    # plant an exact tie later in the store: the lowest index must win
+    store[count - 3] = store[j]
+    am, md = P.nearest(dev(store), dev(q))
+    torch.cuda.synchronize()
+    assert int(am.item()) == O.pose_retrieve(store, q) == j
+    assert abs(float(md.item()) - O.sq_dist(q, store[j])) <= 1e-12 * O.sq_dist(q, store[j])
