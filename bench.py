@@ -266,6 +266,20 @@ def time_attention_kernel(torch, P, wl, stream, reps=10):
     return e0.elapsed_time(e1) / reps / 1e3
 
 
+def max_over_ranks(torch, dist, seconds: float, device) -> float:
+    """Largest per-rank time (all ranks take part; every rank gets the result)."""
+    if dist is None:
+        return seconds
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world: int, steps: int, max_seconds: float) -> float:
+    """Whole-job rounds/s of `world` independent replicas, each doing `steps` rounds."""
+    return world * steps / max_seconds
+
+
 def _event_time(torch, fn, reps, stream):
     with torch.cuda.stream(stream):
         fn()
@@ -390,11 +404,7 @@ def run_ours(args, rank, world, local_rank):
         proc.terminate()
         proc.wait()
         fh.close()
-    elapsed = e0.elapsed_time(e1) / 1e3
-    if dist is not None:
-        t = torch.tensor([elapsed], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(torch, dist, e0.elapsed_time(e1) / 1e3, "cuda")
     if st.device_status(stream) != 0:
         raise RuntimeError("device status word set during the timed region")
 
@@ -426,11 +436,7 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         f1.record(stream)
     barrier()
-    e2e_elapsed = f0.elapsed_time(f1) / 1e3
-    if dist is not None:
-        t = torch.tensor([e2e_elapsed], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_elapsed = float(t.item())
+    e2e_elapsed = max_over_ranks(torch, dist, f0.elapsed_time(f1) / 1e3, "cuda")
 
     # dominant kernel, timed alone on the stream it is launched on
     attn_s = time_attention_kernel(torch, P, wl, stream)
@@ -439,7 +445,7 @@ def run_ours(args, rank, world, local_rank):
     achieved = attn_fl / attn_s / 1e12
 
     launches_per_round = 1 + 7 * len(S.LAYERS) + 3 + 3
-    value = world * args.steps / elapsed
+    value = job_rate(world, args.steps, elapsed)
     line = {
         "metric": METRIC, "value": value, "unit": "rounds/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
@@ -460,7 +466,7 @@ def run_ours(args, rank, world, local_rank):
                      "kernel": "attn_kernel<40> (64x64 level, KV own + bank x4)",
                      "peak_kind": f"{peak_kind} bf16 burst (fp16 dense rate is the same)",
                      "launch_ms": attn_s * 1e3},
-        "e2e": {"value": world * e2e_steps / e2e_elapsed, "unit": "rounds/s",
+        "e2e": {"value": job_rate(world, e2e_steps, e2e_elapsed), "unit": "rounds/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_round * args.steps,
     }
