@@ -452,13 +452,10 @@ template <int HD>
 constexpr int kVar = (HD <= 64) ? 2 : 0;
 constexpr int kExpMode = 0;   // exp2 on the MUFU pipe only
 
-// head_dim 40 and 64 run the transposed-PV kernel (attn_t.cu)
-constexpr bool kTransposedSmallHd = false;
-
 int block_n(int head_dim) {
   switch (head_dim) {
-    case 40: return kTransposedSmallHd ? attn_t_block_n() : Cfg<40, kVar<40>>::BN;
-    case 64: return kTransposedSmallHd ? attn_t_block_n() : Cfg<64, kVar<64>>::BN;
+    case 40: return Cfg<40, kVar<40>>::BN;
+    case 64: return Cfg<64, kVar<64>>::BN;
     case 80: return Cfg<80, kVar<80>>::BN;
     case 128: return Cfg<128, kVar<128>>::BN;
     case 160: return Cfg<160, kVar<160>>::BN;
@@ -553,7 +550,6 @@ int attn_init() {
   if (!done) {
     if (set_attr<40>() || set_attr<64>() || set_attr<80>() || set_attr<128>() || set_attr<160>())
       return 4;
-    if (kTransposedSmallHd && attn_t_init()) return 4;
     done = 1;
   }
   return 0;
@@ -561,8 +557,6 @@ int attn_init() {
 
 int attn_launch(const AttnParams& p, int head_dim, cudaStream_t stream) {
   if (attn_init()) return 4;
-  if (kTransposedSmallHd && (head_dim == 40 || head_dim == 64))
-    return attn_t_launch(p, head_dim, stream);
   switch (head_dim) {
     case 40: return launch_hd<40>(p, stream);
     case 64: return launch_hd<64>(p, stream);

@@ -48,10 +48,6 @@ int attn_make_params(AttnParams* p, const void* q, int64_t ldq, int64_t q_fstrid
                      int head_dim, void* out, int64_t ldo, int64_t out_fstride);
 // Set kernel attributes once (call outside stream capture). 0 on success.
 int attn_init();
-// The transposed-PV kernel for head_dim 40 and 64 (attn_t.cu).
-int attn_t_block_n();
-int attn_t_init();
-int attn_t_launch(const AttnParams& p, int head_dim, cudaStream_t stream);
 int attn_launch(const AttnParams& p, int head_dim, cudaStream_t stream);
 
 }  // namespace pl
