@@ -14,20 +14,20 @@
 // the exact softmax up to rounding.
 //
 // Roles: warpgroup 0 = warp 0 TMA producer (Q once, K/V tiles into a STAGES
-// ring) + warp 1 MMA issuer and TMEM owner (warps 2, 3 idle); warpgroups 1
-// and 2 = softmax of query tiles 0 and 1. setmaxnreg moves registers from
-// warpgroup 0 (120 per thread) to the softmax warpgroups (184 per thread); the
-// launch is refused unless the kernel was compiled at 168 registers per
-// thread, the exact total that split needs. The MMA warp interleaves the two
-// tiles so the tensor pipe works on one tile while the other one's softmax
-// runs.
+// ring), warp 1 MMA issuer of query tile 0 and TMEM owner, warp 2 MMA issuer
+// of query tile 1 when each tile has two S buffers (else warp 1 issues both;
+// warp 3 idle); warpgroups 1 and 2 = softmax of query tiles 0 and 1.
+// setmaxnreg moves registers from warpgroup 0 (120 per thread) to the softmax
+// warpgroups (184 per thread); the launch is refused unless the kernel was
+// compiled at 168 registers per thread, the exact total that split needs.
 //
 // The softmax is issue- and MUFU-bound (one exp2 per score at head_dim 40
 // against 160 tensor FLOPs), so its inner loop uses packed f32x2 FMAs,
 // 3-input max and one of two exp2 paths (EXPM): 0 = ex2.approx.f32 on the
 // MUFU pipe; 2 = MUFU for 3 of every 4 pairs and a degree-3 polynomial
 // on the FMA pipe for the 4th (Cody-Waite split 2^x = 2^n 2^f with n the
-// nearest integer, f in [-0.5, 0.5]; coefficients from exp2_poly.py).
+// nearest integer, f in [-0.5, 0.5]; the cubic is fitted to 2^f on that
+// interval, max relative error 7.7e-5).
 // Measured on B200 (level-64 kernel): ex2.approx.f32 issues 16 results per
 // clock per SM and ex2.approx.f16x2 only 8 instructions (the same 16 results),
 // so the f16x2 path was dropped; the polynomial split (EXPM 2) was 7% slower
@@ -71,6 +71,8 @@ struct Cfg {
   static constexpr size_t SMEM = Q_BYTES + STAGES * STAGE_BYTES + 1024 + 512;
   static_assert(2 * SB * BN + 2 * HDP <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
+  // barriers, TMEM slot, abort flag and segment lengths fit the 512-byte tail
+  static_assert(8 * (18 + 2 * STAGES + 2 * SB) + 8 + 4 * kAttnMaxSegs <= 512, "barrier area");
 };
 
 constexpr int kThreads = 384;
@@ -92,10 +94,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   uint64_t* kv_empty = kv_full + C::STAGES;
   uint64_t* s_full = kv_empty + C::STAGES;   // [2 tiles][SB]
   uint64_t* p_full = s_full + 2 * C::SB;     // [2 tiles][2]
-  uint64_t* o_full = p_full + 4;             // [2 tiles], one phase per PV
+  uint64_t* o_full = p_full + 4;             // [2 tiles]: one phase per PV (one S buffer) or
+                                             // one phase for the next-to-last PV (two S buffers)
   uint64_t* o_final = o_full + 2;            // [2 tiles], one phase: the tile's last PV done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 2);
+  uint64_t* stagger = o_final + 2;           // one phase: tile 0 has reached its first exps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stagger + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // segment lengths, copied once from the parameter space (a constant-cache
+  // miss costs several hundred clocks on a warp's critical path)
+  int* seg_len = reinterpret_cast<int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -123,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     mbar_init(q_full, 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], C::SB == 2 ? 2 : 1);   // one commit per MMA issuer
     }
     for (int b = 0; b < 2 * C::SB; ++b) mbar_init(&s_full[b], 1);
     for (int b = 0; b < 4; ++b) mbar_init(&p_full[b], 128);
@@ -131,6 +138,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       mbar_init(&o_full[i], 1);
       mbar_init(&o_final[i], 1);
     }
+    mbar_init(stagger, 128);
+    for (int sg = 0; sg < n_active; ++sg) seg_len[sg] = p.seg[sg].len;
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -188,8 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || (C::SB == 2 && warp == 2)) {
+    // ------------------------------------------------------------ MMA issuer(s)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_f16_f32(128, C::BN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_f16_f32(128, C::HDP, 0, 1);
@@ -212,14 +221,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         mma_commit(&s_full[i * C::SB + b]);
       };
       // O_i (+)= P_i V with P read from S buffer b (fp16, two keys per column)
-      auto issue_pv = [&](int i, int stage, int b, bool acc) {
+      auto issue_pv = [&](int i, int stage, int b, bool acc, bool commit_o = true) {
         const uint64_t v0 = dv + ((stage * C::STAGE_BYTES) >> 4);
         const uint32_t d = tmem + o_col(i);
         const uint32_t a = tmem + s_col(i, b);
 #pragma unroll
         for (int k = 0; k < C::BN / 16; ++k)
           mma_ts(d, a + k * 8, v0 + ((k * 2048) >> 4), idesc_pv, (acc || k > 0) ? 1u : 0u);
-        mma_commit(&o_full[i]);
+        if (commit_o) mma_commit(&o_full[i]);
       };
       auto wait_p = [&](int i, int jt) {
         const bool r = mbar_wait(&p_full[i * 2 + (jt & 1)], (jt >> 1) & 1, abort_flag);
@@ -231,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       // the MMA side only needs the total tile count (the tiles' segments
       // matter to the producer and the softmax)
       int nt_total = 0;
-      for (int sg = 0; sg < n_active; ++sg) nt_total += (p.seg[sg].len + C::BN - 1) / C::BN;
+      for (int sg = 0; sg < n_active; ++sg) nt_total += (seg_len[sg] + C::BN - 1) / C::BN;
       int stage = 0;
       uint32_t phase = 0;
       auto next_stage = [&]() {
@@ -241,34 +250,41 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
       };
       if constexpr (C::SB == 2) {
-        // S(j) of both tiles first, then the PVs of the previous tile: the
-        // softmax finds S(j) ready when it finishes P(j - 1). (Issuing QK1(j)
-        // after PV0(j - 1) to stagger the two warpgroups measured 3% slower.)
-        int prev_stage = 0;
-        int jt = 0;
-        for (; ok && jt < nt_total; ++jt) {
-          if (!(ok = mbar_wait(&kv_full[stage], phase, abort_flag))) break;
+        // Two issuers: warp 1 runs query tile 0's MMAs and warp 2 tile 1's.
+        // A shared-memory access by an issuing thread (an mbarrier wait
+        // included) is ordered behind the MMAs it has queued, so each wait
+        // lets that thread's queue run dry; with two independent issuers the
+        // tensor pipe executes one tile's MMAs while the other's issuer waits
+        // (measured on B200: 18 MMAs of this shape per KV tile in ~1100
+        // clocks with two issuers against ~1900 with one).
+        // Each tile's S runs two KV tiles ahead of its PV: PV_i(j) frees the
+        // S buffer that QK_i(j + 2) fills. PV completion needs no commit of
+        // its own: S_i(j + 2) landing implies PV_i(j) has (one issuer, in-order
+        // pipe), which is what the softmax waits on before a rescale; only the
+        // next-to-last PV, which no QK follows, commits o_full. A K/V stage is
+        // released by both issuers' commits.
+        static_assert(C::STAGES >= 3, "three KV tiles are in flight");
+        const int i = warp - 1;
+        auto stage_of = [](int t) { return t % C::STAGES; };
+        auto wait_kv = [&](int t) {
+          const bool r = mbar_wait(&kv_full[stage_of(t)], (t / C::STAGES) & 1, abort_flag);
           tc_fence_after();
-          issue_qk(0, stage, jt & 1);
-          issue_qk(1, stage, jt & 1);
-          if (jt > 0) {
-            if (!(ok = wait_p(0, jt - 1))) break;
-            issue_pv(0, prev_stage, (jt - 1) & 1, jt - 1 > 0);
-            if (!(ok = wait_p(1, jt - 1))) break;
-            issue_pv(1, prev_stage, (jt - 1) & 1, jt - 1 > 0);
-            mma_commit(&kv_empty[prev_stage]);
-          }
-          prev_stage = stage;
-          next_stage();
+          return r;
+        };
+        for (int t = 0; ok && t < 2 && t < nt_total; ++t) {
+          if (!(ok = wait_kv(t))) break;
+          issue_qk(i, stage_of(t), t);
         }
-        if (ok && jt > 0 && wait_p(0, jt - 1)) {
-          issue_pv(0, prev_stage, (jt - 1) & 1, jt - 1 > 0);
-          mma_commit(&o_final[0]);
-          if (wait_p(1, jt - 1)) {
-            issue_pv(1, prev_stage, (jt - 1) & 1, jt - 1 > 0);
-            mma_commit(&o_final[1]);
-            mma_commit(&kv_empty[prev_stage]);
-          }
+        for (int jt = 0; ok && jt < nt_total; ++jt) {
+          const int st = stage_of(jt);
+          const int b = jt & 1;
+          const bool ahead = jt + 2 < nt_total;
+          if (!(ok = wait_p(i, jt))) break;
+          if (ahead && !(ok = wait_kv(jt + 2))) break;
+          issue_pv(i, st, b, jt > 0, jt == nt_total - 2);
+          if (jt == nt_total - 1) mma_commit(&o_final[i]);
+          mma_commit(&kv_empty[st]);
+          if (ahead) issue_qk(i, stage_of(jt + 2), b);
         }
       } else {
         int prev_stage = 0;
@@ -314,8 +330,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     float m_run = -INFINITY, l_run = 0.f;
     int jt = 0;
     bool ok = true;
+    // With two S buffers the two tiles' S supplies are independent, so
+    // warpgroup 1 starts its first tile only when warpgroup 0 begins its
+    // first exps: the warpgroups' exp phases then start out of step and
+    // interleave on the MUFU for the first KV tiles instead of coinciding
+    // (measured 3% faster over a level-64 launch; in steady state the two
+    // drift back into step).
+    int nt_all = 0;
+    for (int sg = 0; sg < n_active; ++sg) nt_all += (seg_len[sg] + C::BN - 1) / C::BN;
+    if (C::SB == 2 && i == 1 && n_active > 0) ok = mbar_wait(stagger, 0, abort_flag);
     for (int sg = 0; ok && sg < n_active; ++sg) {
-      const int len = p.seg[sg].len;
+      const int len = seg_len[sg];
       const int nt = (len + C::BN - 1) / C::BN;
       for (int lt = 0; lt < nt; ++lt) {
         const int b = C::SB == 2 ? (jt & 1) : 0;
@@ -354,8 +379,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
         l_run *= alpha;
         if (__any_sync(0xffffffffu, need && jt > 0)) {
-          // rescale O_i once PV(jt - 1) has landed in it
-          if (!(ok = mbar_wait(&o_full[i], (jt - 1) & 1, abort_flag))) break;
+          // rescale O_i once PV(jt - 1) has landed in it: with two S buffers
+          // S_i(jt + 1) is issued after PV_i(jt - 1), so its barrier serves
+          // (the softmax waits on that phase next anyway); PV(nt - 2) has its
+          // own one-shot phase on o_full
+          if constexpr (C::SB == 2) {
+            const bool via_s = jt + 1 < nt_all;
+            ok = via_s ? mbar_wait(&s_full[i * C::SB + ((jt + 1) & 1)], ((jt + 1) >> 1) & 1, abort_flag)
+                       : mbar_wait(&o_full[i], 0, abort_flag);
+          } else {
+            ok = mbar_wait(&o_full[i], (jt - 1) & 1, abort_flag);
+          }
+          if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int c0 = 0; c0 < C::HDP; c0 += 16) {
@@ -368,6 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           }
           tmem_wait_st();
         }
+        if (C::SB == 2 && i == 0 && jt == 0) mbar_arrive(stagger);
         const uint64_t sc2 = f2_pack(sl2, sl2);
         const uint64_t nm2 = f2_pack(-m_run, -m_run);
         float sum = 0.f;
