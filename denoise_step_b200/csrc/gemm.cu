@@ -3,9 +3,14 @@
 //   warp 0      TMA producer: A tile [128 x 64] (K-major) + B tile [64 x BN]
 //               (MN-major, BN/64 column blocks), 128-byte swizzle, STAGES ring
 //   warp 1      MMA issuer (one lane): 4 x tcgen05.mma (K = 16) per stage into
-//               a TMEM accumulator; two accumulators alternate between tiles
+//               a TMEM accumulator; two accumulators alternate between tiles.
+//               It waits for two stages at a time: a wait by the issuing
+//               thread is ordered behind the MMAs it has queued, so each one
+//               lets the tensor pipe run dry for a moment.
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
-//               row), fp32 -> fp16, 16-byte stores
+//               row, 32 columns at a time), fp32 -> fp16 (or kept fp32) into a
+//               swizzled shared-memory chunk of 32 rows x 32 columns, written
+//               out by a TMA tile store (two chunks in flight per warp)
 #include <cuda_runtime.h>
 
 #include "gemm.cuh"
@@ -16,7 +21,7 @@ namespace pl {
 
 namespace {
 
-constexpr int kStages = 5;
+constexpr int kStages = 4;
 constexpr int kNB = (kGemmBN + 63) / 64;            // 64-column B blocks per tile
 constexpr uint32_t kABytes = kGemmBM * 128;          // 128 rows x 128 B
 constexpr uint32_t kBBlockBytes = 64 * 128;          // 64 K-rows x 128 B
@@ -24,7 +29,10 @@ constexpr uint32_t kBBytes = kNB * kBBlockBytes;
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kAccStride = 256;                 // TMEM columns per accumulator
 constexpr int kThreads = 192;
-constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr uint32_t kChunkBytes = 32 * 128;           // 32 rows x 32 columns, fp32 worst case
+constexpr uint32_t kStagingBytes = 4 * 2 * kChunkBytes;   // 4 epilogue warps x 2 chunks
+constexpr size_t kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + 256;
+static_assert(kGemmBN % 32 == 0, "32-column epilogue chunks");
 
 struct TileCoord {
   int prob, m0, n0;
@@ -46,7 +54,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* staging = smem + kStages * kStageBytes;     // 1024-byte aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + kStagingBytes);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
@@ -123,18 +132,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
         if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t d = tmem + buf * kAccStride;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < nk; kb += 2) {
+          const bool two = kb + 1 < nk;
+          // both stages' waits back to back, then their 8 MMAs in one burst
           if (!mbar_wait(&full[stage], phase, abort_flag)) break;
+          const int stage2 = stage + 1 == kStages ? 0 : stage + 1;
+          const uint32_t phase2 = stage + 1 == kStages ? phase ^ 1 : phase;
+          if (two && !mbar_wait(&full[stage2], phase2, abort_flag)) break;
           tc_fence_after();
-          const uint64_t ad = da + ((stage * kStageBytes) >> 4);
-          const uint64_t bd = db + ((stage * kStageBytes) >> 4);
 #pragma unroll
-          for (int k = 0; k < kGemmBK / 16; ++k)
-            mma_ss(d, ad + ((32 * k) >> 4), bd + ((2048 * k) >> 4), idesc, (kb > 0 || k > 0) ? 1u : 0u);
-          mma_commit(&empty[stage]);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1;
+          for (int h = 0; h < 2; ++h) {
+            if (h == 1 && !two) break;
+            const int sth = h == 0 ? stage : stage2;
+            const uint64_t ad = da + ((sth * kStageBytes) >> 4);
+            const uint64_t bd = db + ((sth * kStageBytes) >> 4);
+#pragma unroll
+            for (int k = 0; k < kGemmBK / 16; ++k)
+              mma_ss(d, ad + ((32 * k) >> 4), bd + ((2048 * k) >> 4), idesc,
+                     (kb + h > 0 || k > 0) ? 1u : 0u);
+            mma_commit(&empty[sth]);
+          }
+          const int adv = two ? 2 : 1;
+          for (int a = 0; a < adv; ++a) {
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
         }
         mma_commit(&acc_full[buf]);
@@ -144,8 +167,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
     __syncwarp();
   } else {
     const int q = warp & 3;   // TMEM lane quadrant this warp may access
-    const int row_in_tile = 32 * q + lane;
+    uint8_t* stg = staging + q * 2 * kChunkBytes;
     int acc_i = 0;
+    int n_chunk = 0;          // chunks this warp has stored (staging slot = n_chunk & 1)
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
       TileCoord tc;
       if (!decode_tile(p, t, tc)) continue;
@@ -154,41 +178,55 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
       const uint32_t use = static_cast<uint32_t>(acc_i >> 1);
       if (!mbar_wait(&acc_full[buf], use & 1, abort_flag)) break;
       tc_fence_after();
-      const int row = tc.m0 + row_in_tile;
       const uint32_t taddr = tmem + buf * kAccStride + (static_cast<uint32_t>(32 * q) << 16);
-      __half* crow = static_cast<__half*>(pr.c) + static_cast<int64_t>(row) * pr.ldc;
-      float* frow = static_cast<float*>(pr.c) + static_cast<int64_t>(row) * pr.ldc;
+      const int y = tc.m0 + 32 * q;
+      const bool rows_in = y < pr.M;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kGemmBN; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(taddr + c0, r);
+      for (int c0 = 0; c0 < kGemmBN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(taddr + c0, r);
         tmem_wait_ld();
-        const int col = tc.n0 + c0;
-        if (row < pr.M && col < pr.N && pr.out_f32) {
-          float4* dst = reinterpret_cast<float4*>(frow + col);
-#pragma unroll
-          for (int q4i = 0; q4i < 4; ++q4i)
-            dst[q4i] = make_float4(__uint_as_float(r[4 * q4i]), __uint_as_float(r[4 * q4i + 1]),
-                                   __uint_as_float(r[4 * q4i + 2]), __uint_as_float(r[4 * q4i + 3]));
-        } else if (row < pr.M && col < pr.N) {
-          uint4 v0, v1;
-          v0.x = pack_half2(__uint_as_float(r[0]), __uint_as_float(r[1]));
-          v0.y = pack_half2(__uint_as_float(r[2]), __uint_as_float(r[3]));
-          v0.z = pack_half2(__uint_as_float(r[4]), __uint_as_float(r[5]));
-          v0.w = pack_half2(__uint_as_float(r[6]), __uint_as_float(r[7]));
-          v1.x = pack_half2(__uint_as_float(r[8]), __uint_as_float(r[9]));
-          v1.y = pack_half2(__uint_as_float(r[10]), __uint_as_float(r[11]));
-          v1.z = pack_half2(__uint_as_float(r[12]), __uint_as_float(r[13]));
-          v1.w = pack_half2(__uint_as_float(r[14]), __uint_as_float(r[15]));
-          uint4* dst = reinterpret_cast<uint4*>(crow + col);
-          dst[0] = v0;
-          dst[1] = v1;
+        if (c0 + 32 >= kGemmBN) {
+          // the accumulator is free once its last columns are in registers
+          tc_fence_before();
+          mbar_arrive(&acc_empty[buf]);
         }
+        const int x = tc.n0 + c0;
+        if (!rows_in || x >= pr.N) continue;
+        // the slot's previous store must have finished reading it
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        uint8_t* chunk = stg + (n_chunk & 1) * kChunkBytes;
+        if (pr.out_f32) {
+          // 128-byte rows, 16-byte unit j of row `lane` at j ^ (lane & 7)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(chunk + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+        } else {
+          // 64-byte rows, 16-byte unit j of row `lane` at j ^ ((lane >> 1) & 3)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 v;
+            v.x = pack_half2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+            v.y = pack_half2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+            v.z = pack_half2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+            v.w = pack_half2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+            *reinterpret_cast<uint4*>(chunk + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) = v;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&pr.c, chunk, x, y);
+          bulk_commit_group();
+        }
+        ++n_chunk;
       }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[buf]);
       ++acc_i;
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -223,8 +261,12 @@ int gemm_make_problem(GemmProblem* p, const void* a, int64_t lda, const void* b,
     const uint32_t box[2] = {64, 64};
     if (encode_f16_tmap(&p->b, b, 2, dims, strides, box) != 0) return 2;
   }
-  p->c = c;
-  p->ldc = ldc;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(M)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(ldc) * (out_f32 ? 4 : 2)};
+    const uint32_t box[2] = {32, 32};
+    if (encode_tmap(&p->c, out_f32, c, 2, dims, strides, box, out_f32 ? 128 : 64) != 0) return 2;
+  }
   p->out_f32 = out_f32 ? 1 : 0;
   p->M = M;
   p->N = N;

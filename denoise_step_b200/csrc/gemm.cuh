@@ -18,8 +18,8 @@ constexpr int kGemmMaxProblems = 16;
 struct GemmProblem {
   CUtensorMap a;        // 2D {K, M}, box {64, 128}, 128B swizzle (K-major A)
   CUtensorMap b;        // 2D {N, K}, box {64, 64}, 128B swizzle (MN-major B)
-  void* c;                    // fp16, or fp32 when out_f32
-  int64_t ldc;                // elements
+  CUtensorMap c;        // 2D {N, M}, box {32, 32}: fp16 with 64-byte swizzle or
+                        // fp32 (out_f32) with 128-byte swizzle; stored by TMA
   int out_f32;
   int M, N, K;
   int tiles_n;

@@ -20,8 +20,8 @@ static void load_encode() {
   }
 }
 
-int encode_f16_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                    const uint64_t* strides_bytes, const uint32_t* box) {
+int encode_tmap(CUtensorMap* m, bool f32, const void* base, int rank, const uint64_t* dims,
+                const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes) {
   std::call_once(g_encode_once, load_encode);
   if (!g_encode) return -1;
   cuuint64_t gdim[5];
@@ -34,11 +34,20 @@ int encode_f16_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* 
     estride[i] = 1;
   }
   for (int i = 0; i < rank - 1; ++i) gstride[i] = strides_bytes[i];
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, static_cast<cuuint32_t>(rank),
-                        const_cast<void*>(base), gdim, gstride, bdim, estride,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (swizzle_bytes == 64) sw = CU_TENSOR_MAP_SWIZZLE_64B;
+  else if (swizzle_bytes == 32) sw = CU_TENSOR_MAP_SWIZZLE_32B;
+  else if (swizzle_bytes != 128) return -2;
+  CUresult r = g_encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        static_cast<cuuint32_t>(rank), const_cast<void*>(base), gdim, gstride, bdim,
+                        estride, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return static_cast<int>(r);
+}
+
+int encode_f16_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box) {
+  return encode_tmap(m, false, base, rank, dims, strides_bytes, box, 128);
 }
 
 }  // namespace pl

@@ -11,5 +11,8 @@ namespace pl {
 // Returns 0 on success, a CUresult (or -1 when the entry point is missing).
 int encode_f16_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box);
+// Same for fp16 or fp32 elements and a 32-, 64- or 128-byte swizzle.
+int encode_tmap(CUtensorMap* m, bool f32, const void* base, int rank, const uint64_t* dims,
+                const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
 
 }  // namespace pl
