@@ -15,8 +15,9 @@
 //
 // Roles: warpgroup 0 = warp 0 TMA producer (Q once, K/V tiles into a STAGES
 // ring), warp 1 MMA issuer of query tile 0 and TMEM owner, warp 2 MMA issuer
-// of query tile 1 when each tile has two S buffers (else warp 1 issues both;
-// warp 3 idle); warpgroups 1 and 2 = softmax of query tiles 0 and 1.
+// of query tile 1 when each tile has two S buffers (else warp 1 issues both,
+// which measured faster there; warp 3 idle); warpgroups 1 and 2 = softmax of
+// query tiles 0 and 1.
 // setmaxnreg moves registers from warpgroup 0 (120 per thread) to the softmax
 // warpgroups (184 per thread); the launch is refused unless the kernel was
 // compiled at 168 registers per thread, the exact total that split needs.
@@ -481,11 +482,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   if (threadIdx.x == 0 && *abort_flag && p.status) atomicOr(p.status, DEV_TIMEOUT);
 }
 
-// Tile schedule per head dimension (measured on B200, level-64 shape): 96-key
-// tiles with two S buffers per query tile where TMEM holds them (head_dim <=
-// 64), 128-key tiles with one S buffer otherwise (64 keys at head_dim 160).
+// Tile schedule per head dimension (measured on B200 with the two MMA
+// issuers): 96-key tiles with two S buffers per query tile where TMEM holds
+// them (head_dim <= 64), 64-key tiles with two S buffers up to head_dim 128
+// (level-32 layer 0.355 -> 0.303 ms against 128-key single-buffered tiles,
+// PR-Sink block 2.02 -> 1.94 ms), 64-key single-buffered tiles with one
+// issuer at head_dim 160.
 template <int HD>
-constexpr int kVar = (HD <= 64) ? 2 : 0;
+constexpr int kVar = (HD <= 64) ? 2 : (HD <= 128 ? 1 : 0);
 constexpr int kExpMode = 0;   // exp2 on the MUFU pipe only
 
 int block_n(int head_dim) {
