@@ -39,12 +39,22 @@ __device__ __forceinline__ int t_index(int t) {  // 999 -> 0, 666 -> 1, 333 -> 2
 
 // ------------------------------------------------------------------ prefill
 // 3 windows at t = 0, 333, 666 (oldest first) in slots 0..2; slot 3 free.
+// blockIdx.z = session (every buffer carries a leading session dimension).
 __global__ void prefill_kernel(DevState* st, float* ring, float* slot_motion, float* bank,
                                const float* __restrict__ ref_latent,
                                const float* __restrict__ prefill_eps,
                                const float* __restrict__ ref_motion,
                                const float* __restrict__ drive0, int64_t frame_elems,
-                               DdimCoef coef) {
+                               int capacity, DdimCoef coef) {
+  const int z = blockIdx.z;
+  st += z;
+  ring += z * 16 * frame_elems;
+  slot_motion += z * 16 * 512;
+  bank += static_cast<int64_t>(z) * capacity * 512;
+  ref_latent += z * frame_elems;
+  prefill_eps += z * 12 * frame_elems;
+  ref_motion += z * 512;
+  drive0 += z * 512;
   const int64_t total = 12 * frame_elems;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -85,9 +95,17 @@ __global__ void prefill_kernel(DevState* st, float* ring, float* slot_motion, fl
 }
 
 // ------------------------------------------------------------------ ring push
+// blockIdx.z = session.
 __global__ void ring_push_kernel(DevState* st, float* ring, float* slot_motion,
                                  float* batch_motion, const float* __restrict__ new_noise,
                                  const float* __restrict__ new_motion, int64_t frame_elems) {
+  const int z = blockIdx.z;
+  st += z;
+  ring += z * 16 * frame_elems;
+  slot_motion += z * 16 * 512;
+  batch_motion += z * 16 * 512;
+  new_noise += z * 4 * frame_elems;
+  new_motion += z * 4 * 512;
   const int head = st->head;
   const int slot = (head + 3) & 3;
   const int64_t n4 = 4 * frame_elems / 4;
@@ -120,11 +138,16 @@ __global__ void ring_push_kernel(DevState* st, float* ring, float* slot_motion,
 
 // ------------------------------------------------------------------ DDIM
 // Batch frame f = blockIdx.y belongs to window w = f / 4 (oldest first), in
-// physical slot (head + w) & 3. Arithmetic in fp64 (x0 via the precomputed
-// 1/sqrt(abar_t)), one rounding to fp32 per output.
+// physical slot (head + w) & 3; blockIdx.z = session. Arithmetic in fp64 (x0
+// via the precomputed 1/sqrt(abar_t)), one rounding to fp32 per output.
 __global__ void ddim_kernel(const DevState* __restrict__ st, float* ring,
                             const float* __restrict__ eps, float* __restrict__ out_x0,
                             int64_t frame_elems, DdimCoef coef) {
+  const int z = blockIdx.z;
+  st += z;
+  ring += z * 16 * frame_elems;
+  eps += z * 16 * frame_elems;
+  out_x0 += z * 4 * frame_elems;
   const int f = blockIdx.y;
   const int w = f >> 2, j = f & 3;
   const int slot = (st->head + w) & 3;
@@ -154,7 +177,9 @@ __global__ void ddim_kernel(const DevState* __restrict__ st, float* ring,
   }
 }
 
+// one block per session
 __global__ void ring_commit_kernel(DevState* st) {
+  st += blockIdx.x;
   int popped = 0;
   for (int s = 0; s < 4; ++s) {
     const int t = st->slot_t[s];
@@ -183,6 +208,18 @@ __global__ void __launch_bounds__(kBankThreads) bank_check_kernel(
   __shared__ int s_cnt, s_app, s_do_append;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int nwarps = kBankThreads / 32;
+  if (st) {
+    // one block per session: its bank, queries, results and state
+    const int z = blockIdx.x;
+    st += z;
+    count_p = &st->bank_count;
+    appends_p = &st->appends;
+    bank += static_cast<int64_t>(z) * capacity * dim;
+    queries += static_cast<int64_t>(z) * nq * dim;
+    if (argmin) argmin += z * nq;
+    if (min_d2) min_d2 += z * nq;
+    if (appended) appended += z * nq;
+  }
   if (threadIdx.x == 0) {
     s_cnt = count_p ? *count_p : count_val;
     s_app = appends_p ? *appends_p : 0;
@@ -279,10 +316,110 @@ __global__ void motion_kv_kernel(const float* __restrict__ motion, const __half*
   }
 }
 
-// One thread per (query row, head): 32 scores in registers, smem-resident
-// K/V of the frame and head (fp32), softmax in fp32.
+// One thread per R = 2 query rows (n, n + 128) of one head: R x 32 scores in
+// registers, K/V of the frame and head in shared memory (fp32), softmax in
+// fp32. Every 16-byte shared-memory read of K or V feeds both rows. Used up
+// to head_dim 64 (64x64 layer: whole cross-attention 182 -> 171 us); at
+// larger head dims its register cost and halved grid measured slower than
+// the one-row kernel below.
+constexpr int kMotionRows = 2;
+
 template <int HD>
 __global__ void __launch_bounds__(128) motion_attn_kernel(const float* __restrict__ q, int64_t ldq,
+                                                          const float* __restrict__ kv, int N,
+                                                          int C, __half* __restrict__ out,
+                                                          int64_t ldo, float scale) {
+  static_assert(HD % 8 == 0, "head_dim");
+  constexpr int R = kMotionRows;
+  __shared__ __align__(16) float sk[32][HD];
+  __shared__ __align__(16) float sv[32][HD];
+  const int f = blockIdx.z, h = blockIdx.y;
+  const float* kvf = kv + static_cast<int64_t>(f) * 32 * 2 * C;
+  for (int i = threadIdx.x; i < 32 * HD; i += blockDim.x) {
+    const int p = i / HD, d = i % HD;
+    sk[p][d] = kvf[p * 2 * C + h * HD + d];
+    sv[p][d] = kvf[p * 2 * C + C + h * HD + d];
+  }
+  __syncthreads();
+  const int n0 = blockIdx.x * 128 * R + threadIdx.x;
+  if (n0 >= N) return;
+  const float* qr[R];
+  bool has[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    has[r] = n0 + 128 * r < N;
+    qr[r] = q + (static_cast<int64_t>(f) * N + (has[r] ? n0 + 128 * r : n0)) * ldq + h * HD;
+  }
+  float s[R][32];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int j = 0; j < 32; ++j) s[r][j] = 0.f;
+#pragma unroll
+  for (int d0 = 0; d0 < HD; d0 += 4) {
+    float4 a[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) a[r] = *reinterpret_cast<const float4*>(qr[r] + d0);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float4 k = *reinterpret_cast<const float4*>(&sk[j][d0]);
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        s[r][j] = fmaf(a[r].x, k.x, fmaf(a[r].y, k.y, fmaf(a[r].z, k.z, fmaf(a[r].w, k.w, s[r][j]))));
+    }
+  }
+  float inv[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      s[r][j] *= scale;
+      m = fmaxf(m, s[r][j]);
+    }
+    float l = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      s[r][j] = __expf(s[r][j] - m);
+      l += s[r][j];
+    }
+    inv[r] = 1.f / l;
+  }
+  __half* orow = out + (static_cast<int64_t>(f) * N + n0) * ldo + h * HD;
+#pragma unroll
+  for (int d0 = 0; d0 < HD; d0 += 8) {
+    float o[R][8];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[r][e] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float4 va = *reinterpret_cast<const float4*>(&sv[j][d0]);
+      const float4 vb = *reinterpret_cast<const float4*>(&sv[j][d0 + 4]);
+      const float v[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[r][e] = fmaf(s[r][j], v[e], o[r][e]);
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (!has[r]) continue;
+      uint4 w;
+      w.x = pack_half2(o[r][0] * inv[r], o[r][1] * inv[r]);
+      w.y = pack_half2(o[r][2] * inv[r], o[r][3] * inv[r]);
+      w.z = pack_half2(o[r][4] * inv[r], o[r][5] * inv[r]);
+      w.w = pack_half2(o[r][6] * inv[r], o[r][7] * inv[r]);
+      *reinterpret_cast<uint4*>(orow + static_cast<int64_t>(128 * r) * ldo + d0) = w;
+    }
+  }
+}
+
+// One thread per (query row, head): 32 scores in registers, smem-resident
+// K/V of the frame and head (fp32), softmax in fp32 (head_dim >= 80).
+template <int HD>
+__global__ void __launch_bounds__(128) motion_attn_row_kernel(const float* __restrict__ q, int64_t ldq,
                                                           const float* __restrict__ kv, int N,
                                                           int C, __half* __restrict__ out,
                                                           int64_t ldo, float scale) {
@@ -471,40 +608,44 @@ int grid_for(int64_t work, int threads) {
 cudaError_t launch_prefill(DevState* st, float* ring, float* slot_motion, float* bank,
                            const float* ref_latent, const float* prefill_eps,
                            const float* ref_motion, const float* drive0, int64_t frame_elems,
-                           cudaStream_t s) {
+                           int capacity, int sessions, cudaStream_t s) {
   DdimCoef coef;
   ddim_coefficients(&coef);
-  prefill_kernel<<<grid_for(12 * frame_elems, 256), 256, 0, s>>>(
-      st, ring, slot_motion, bank, ref_latent, prefill_eps, ref_motion, drive0, frame_elems, coef);
+  const dim3 grid(static_cast<unsigned>(grid_for(12 * frame_elems, 256)), 1, sessions);
+  prefill_kernel<<<grid, 256, 0, s>>>(st, ring, slot_motion, bank, ref_latent, prefill_eps,
+                                      ref_motion, drive0, frame_elems, capacity, coef);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ring_push(DevState* st, float* ring, float* slot_motion, float* batch_motion,
                              const float* new_noise, const float* new_motion,
-                             int64_t frame_elems, cudaStream_t s) {
-  ring_push_kernel<<<grid_for(frame_elems, 256), 256, 0, s>>>(st, ring, slot_motion, batch_motion,
-                                                             new_noise, new_motion, frame_elems);
+                             int64_t frame_elems, int sessions, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>(grid_for(frame_elems, 256)), 1, sessions);
+  ring_push_kernel<<<grid, 256, 0, s>>>(st, ring, slot_motion, batch_motion, new_noise, new_motion,
+                                        frame_elems);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ddim(DevState* st, float* ring, const float* eps, float* out_x0,
-                        int64_t frame_elems, const DdimCoef& coef, cudaStream_t s) {
-  dim3 grid(static_cast<unsigned>((grid_for(frame_elems / 4, 256) + 15) / 16), 16);
+                        int64_t frame_elems, const DdimCoef& coef, int sessions, cudaStream_t s) {
+  dim3 grid(static_cast<unsigned>((grid_for(frame_elems / 4, 256) + 15) / 16), 16, sessions);
   ddim_kernel<<<grid, 256, 0, s>>>(st, ring, eps, out_x0, frame_elems, coef);
   return cudaGetLastError();
 }
 
-cudaError_t launch_ring_commit(DevState* st, cudaStream_t s) {
-  ring_commit_kernel<<<1, 1, 0, s>>>(st);
+cudaError_t launch_ring_commit(DevState* st, int sessions, cudaStream_t s) {
+  ring_commit_kernel<<<sessions, 1, 0, s>>>(st);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bank_check(float* bank, int32_t* count, int32_t* appends, int capacity,
                               int dim, const float* queries, int nq, double thr2, int cap,
                               int32_t* argmin, double* min_d2, uint8_t* appended,
-                              DevState* st, cudaStream_t s) {
-  bank_check_kernel<<<1, kBankThreads, 0, s>>>(bank, count, appends, capacity, dim, queries, nq,
-                                               thr2, cap, argmin, min_d2, appended, st, 0);
+                              DevState* st, int sessions, cudaStream_t s) {
+  if (!st && sessions != 1) return cudaErrorInvalidValue;
+  bank_check_kernel<<<sessions, kBankThreads, 0, s>>>(bank, count, appends, capacity, dim, queries,
+                                                      nq, thr2, cap, argmin, min_d2, appended, st,
+                                                      0);
   return cudaGetLastError();
 }
 
@@ -549,14 +690,14 @@ cudaError_t launch_motion_kv(const float* motion, const __half* m_kv, int F, int
 cudaError_t launch_motion_attn(const float* q, int64_t ldq, const float* kv, int F, int N,
                                int C, int heads, __half* out, int64_t ldo, cudaStream_t s) {
   const int hd = C / heads;
-  dim3 grid((N + 127) / 128, heads, F);
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(hd)));
+  auto grid = [&](int rows) { return dim3((N + 128 * rows - 1) / (128 * rows), heads, F); };
   switch (hd) {
-    case 40: motion_attn_kernel<40><<<grid, 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
-    case 64: motion_attn_kernel<64><<<grid, 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
-    case 80: motion_attn_kernel<80><<<grid, 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
-    case 128: motion_attn_kernel<128><<<grid, 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
-    case 160: motion_attn_kernel<160><<<grid, 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
+    case 40: motion_attn_kernel<40><<<grid(kMotionRows), 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
+    case 64: motion_attn_kernel<64><<<grid(kMotionRows), 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
+    case 80: motion_attn_row_kernel<80><<<grid(1), 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
+    case 128: motion_attn_row_kernel<128><<<grid(1), 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
+    case 160: motion_attn_row_kernel<160><<<grid(1), 128, 0, s>>>(q, ldq, kv, N, C, out, ldo, scale); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -5,6 +5,7 @@
     python -m denoise_step_b200.microbench ddim --h 64 --w 64 --reps 3
     python -m denoise_step_b200.microbench sink --n 4096 --c 5120 --heads 40 --pool 64 --reps 3
     python -m denoise_step_b200.microbench nearest --count 1048576 --dim 128 --reps 10
+    python -m denoise_step_b200.microbench motion --frames 16 --n 4096 --c 320 --heads 8 --reps 10
 
 Inputs are seeded torch tensors on the device; prints the mean CUDA-event time
 per launch and the algorithmic throughput.
@@ -91,6 +92,23 @@ def gemm(a, stream):
             "gbs": 2.0 * (a.m * a.k + a.k * a.n + a.m * a.n) / t / 1e9}
 
 
+def motion(a, stream):
+    """Motion cross-attention of one layer: Mq GEMM (fp32 out), 32-token attention, Mo GEMM."""
+    g = torch.Generator(device="cuda").manual_seed(a.seed)
+    F, N, Cc = a.frames, a.n, a.c
+    x = torch.randn((F, N, Cc), device="cuda", dtype=torch.float16, generator=g)
+    mot = torch.randn((F, 512), device="cuda", dtype=torch.float32, generator=g)
+    w = lambda r, c: torch.randn((r, c), device="cuda", dtype=torch.float16, generator=g) / r ** 0.5
+    m_q, m_kv, m_o = w(Cc, Cc), w(16, 2 * Cc), w(Cc, Cc)
+    out = torch.empty_like(x)
+    need = P.sz()
+    P.check(P.lib.pl_motion_xattn_workspace_bytes(F, N, Cc, P.C.byref(need)), "ws")
+    ws = torch.empty(need.value, dtype=torch.uint8, device="cuda")
+    t = _time(lambda: P.motion_xattn(x, mot, m_q, m_kv, m_o, a.heads, out=out, workspace=ws,
+                                     stream=stream), a.reps, stream)
+    return {"kernel": f"motion xattn C{Cc}", "s": t}
+
+
 def ddim(a, stream):
     st = P.Stream(P.make_config((a.h, a.w), []))
     fe = 4 * a.h * a.w
@@ -112,7 +130,7 @@ def ddim(a, stream):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["attn", "gemm", "ddim", "sink", "nearest"])
+    ap.add_argument("what", choices=["attn", "gemm", "ddim", "sink", "nearest", "motion"])
     ap.add_argument("--count", type=int, default=1 << 20)
     ap.add_argument("--dim", type=int, default=128)
     ap.add_argument("--pool", type=int, default=64)
@@ -129,7 +147,8 @@ def main():
     ap.add_argument("--seed", type=int, default=1002)
     a = ap.parse_args()
     stream = torch.cuda.Stream()
-    r = {"attn": attn, "gemm": gemm, "ddim": ddim, "sink": sink, "nearest": nearest}[a.what](a, stream)
+    r = {"attn": attn, "gemm": gemm, "ddim": ddim, "sink": sink, "nearest": nearest,
+         "motion": motion}[a.what](a, stream)
     print(json.dumps(r))
 
 
