@@ -39,7 +39,8 @@ class Config(C.Structure):
     _fields_ = [("latent_c", C.c_int32), ("latent_h", C.c_int32), ("latent_w", C.c_int32),
                 ("n_layers", C.c_int32), ("layer_tokens", C.c_int32 * MAX_LAYERS),
                 ("layer_channels", C.c_int32 * MAX_LAYERS), ("heads", C.c_int32),
-                ("drift_threshold", C.c_float), ("append_cap", C.c_int32)]
+                ("drift_threshold", C.c_float), ("append_cap", C.c_int32),
+                ("sessions", C.c_int32)]
 
 
 class LayerWeights(C.Structure):
@@ -84,7 +85,9 @@ _SIGS = {
     "pl_ctx_bank_check": (i32, [vp, vp, i32, vp, vp, vp, vp]),
     "pl_stream_round": (i32, [vp, vp, vp, C.POINTER(vp), vp, vp, vp, C.POINTER(vp), vp]),
     "pl_get_state": (i32, [vp, C.POINTER(State), vp]),
+    "pl_get_session_state": (i32, [vp, i32, C.POINTER(State), vp]),
     "pl_get_motion_bank": (i32, [vp, vp, C.POINTER(C.c_int32), vp]),
+    "pl_get_session_motion_bank": (i32, [vp, i32, vp, C.POINTER(C.c_int32), vp]),
     "pl_get_device_status": (i32, [vp, vp]),
     "pl_ctx_ring_latents": (vp, [vp]),
 }
@@ -261,8 +264,9 @@ def nearest(store, query, argmin=None, min_d2=None, workspace=None, stream=None)
 
 # --------------------------------------------------------------------------- stream context
 
-def make_config(latent_hw=(64, 64), layers=(), heads=8, threshold=17.0, append_cap=3, latent_c=4):
-    """layers: sequence of (tokens N, channels C)."""
+def make_config(latent_hw=(64, 64), layers=(), heads=8, threshold=17.0, append_cap=3, latent_c=4,
+                sessions=1):
+    """layers: sequence of (tokens N, channels C); sessions: streams served together."""
     cfg = Config()
     cfg.latent_c, (cfg.latent_h, cfg.latent_w) = latent_c, latent_hw
     cfg.n_layers = len(layers)
@@ -272,11 +276,16 @@ def make_config(latent_hw=(64, 64), layers=(), heads=8, threshold=17.0, append_c
     cfg.heads = heads
     cfg.drift_threshold = threshold
     cfg.append_cap = append_cap
+    cfg.sessions = sessions
     return cfg
 
 
 class Stream:
-    """One PersonaLive stream: the device-resident pile and the reference bank."""
+    """PersonaLive stream(s): the device-resident piles and reference banks.
+
+    With cfg.sessions = S > 1 the context serves S independent streams in the
+    same launches; every per-stream tensor argument then has a leading
+    dimension S (session-major, contiguous)."""
 
     def __init__(self, cfg: Config, device="cuda"):
         import torch
@@ -339,17 +348,18 @@ class Stream:
                                   _ptr(out_frames), _ptr(appended), lo, _stream(stream)),
               "pl_stream_round")
 
-    def state(self, stream=None):
+    def state(self, stream=None, session=0):
         s = State()
-        check(lib.pl_get_state(self.handle, C.byref(s), _stream(stream)), "pl_get_state")
+        check(lib.pl_get_session_state(self.handle, session, C.byref(s), _stream(stream)),
+              "pl_get_session_state")
         return s.as_dict()
 
-    def motion_bank(self, stream=None):
+    def motion_bank(self, stream=None, session=0):
         import numpy as np
         buf = np.zeros((4, 512), dtype=np.float32)
         n = C.c_int32()
-        check(lib.pl_get_motion_bank(self.handle, buf.ctypes.data, C.byref(n), _stream(stream)),
-              "pl_get_motion_bank")
+        check(lib.pl_get_session_motion_bank(self.handle, session, buf.ctypes.data, C.byref(n),
+                                             _stream(stream)), "pl_get_session_motion_bank")
         return buf[: n.value].copy()
 
     def device_status(self, stream=None) -> int:

@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 
   int n_active = p.n_total;
   if (p.n_extra != nullptr) {
-    int extra = *((volatile const int32_t*)p.n_extra);
+    const int si = p.extra_div > 0 ? frame / p.extra_div : 0;
+    int extra = *((volatile const int32_t*)(p.n_extra + static_cast<int64_t>(si) * p.extra_stride));
     extra = extra < 0 ? 0 : extra;
     const int avail = p.n_total - p.n_fixed;
     n_active = p.n_fixed + (extra < avail ? extra : avail);
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       uint32_t phase = 0;
       for (int sg = 0; sg < n_active && !*abort_flag; ++sg) {
         const AttnSeg& seg = p.seg[sg];
-        int fr = seg.per_frame ? frame : 0;
+        int fr = seg.per_frame ? frame : (seg.frame_div > 0 ? frame / seg.frame_div : 0);
         if (seg.block_sel != nullptr) {
           fr = *((volatile const int32_t*)seg.block_sel);
           if (fr < 0 || fr >= seg.n_blocks) {   // out of range: attend block 0, flag it
@@ -553,8 +554,12 @@ int attn_make_params(AttnParams* p, const void* q, int64_t ldq, int64_t q_fstrid
       return 1;
     if (h.ld < static_cast<int64_t>(heads) * head_dim) return 1;
     if ((reinterpret_cast<uintptr_t>(h.k) | reinterpret_cast<uintptr_t>(h.v)) & 15) return 1;
-    const bool stacked = h.block_sel != nullptr;
+    const bool stacked = h.block_sel != nullptr || h.frame_div > 0;
+    if (h.block_sel != nullptr && h.frame_div > 0) return 1;
+    if (h.frame_div < 0) return 1;
     if (stacked && (h.n_blocks < 1 || h.frame_stride <= 0)) return 1;
+    // every frame's block must exist
+    if (h.frame_div > 0 && (frames - 1) / h.frame_div >= h.n_blocks) return 1;
     const bool per_frame = !stacked && h.frame_stride != 0 && frames > 1;
     const int64_t fs = (per_frame || stacked) ? h.frame_stride : h.len * h.ld;
     const uint64_t n4 = stacked ? static_cast<uint64_t>(h.n_blocks) : (per_frame ? frames : 1);
@@ -569,10 +574,13 @@ int attn_make_params(AttnParams* p, const void* q, int64_t ldq, int64_t q_fstrid
     p->seg[s].per_frame = per_frame ? 1 : 0;
     p->seg[s].block_sel = h.block_sel;
     p->seg[s].n_blocks = static_cast<int>(n4);
+    p->seg[s].frame_div = h.frame_div;
   }
   p->n_fixed = n_segs;
   p->n_total = n_segs;
   p->n_extra = nullptr;
+  p->extra_div = 0;
+  p->extra_stride = 0;
   p->out = static_cast<__half*>(out);
   p->ldo = ldo;
   p->out_fstride = out_fstride;

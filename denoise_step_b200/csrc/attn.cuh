@@ -16,6 +16,8 @@ struct AttnSeg {
   const int32_t* block_sel;  // when non-null: every frame reads block *block_sel
                              // of a stacked segment (a retrieved cache block)
   int n_blocks;              // blocks in a stacked segment
+  int frame_div;             // when > 0: frame f reads block f / frame_div of a stacked
+                             // segment (one block per session of frame_div frames)
 };
 
 struct AttnParams {
@@ -23,7 +25,9 @@ struct AttnParams {
   AttnSeg seg[kAttnMaxSegs];
   int n_fixed;                 // segments always attended
   int n_total;                 // segments available
-  const int32_t* n_extra;      // when non-null: attend n_fixed + min(*n_extra, n_total - n_fixed)
+  const int32_t* n_extra;      // when non-null: attend n_fixed + min(e, n_total - n_fixed) with
+                               // e = n_extra[(frame / extra_div) * extra_stride]
+  int extra_div, extra_stride; // frames per session and int32 stride between sessions' counts
   __half* out;
   int64_t ldo, out_fstride;
   int n_q, heads, frames;
@@ -40,6 +44,9 @@ struct AttnSegHost {
   // chosen on the device by *block_sel (0 <= *block_sel < n_blocks)
   int64_t n_blocks = 0;
   const int32_t* block_sel = nullptr;
+  // optional: `n_blocks` blocks stacked at `frame_stride`, frame f reading
+  // block f / frame_div (frame_div > 0; excludes block_sel)
+  int frame_div = 0;
 };
 
 // Build params (tensor maps) on the host. Returns 0 on success.

@@ -21,6 +21,10 @@ struct DevState {
   uint32_t status;
   uint32_t pad2_[3];
 };
+// States of several sessions sit in an array; kernels step through it by
+// whole int32 words (the attention reads appends at a fixed word stride).
+static_assert(sizeof(DevState) % sizeof(int32_t) == 0 && sizeof(DevState) % 8 == 0,
+              "DevState array stride");
 
 // Per-timestep DDIM coefficients for the 4 timesteps of the table, in table
 // order t = 999, 666, 333, 0: c = {1/sqrt(abar_t), sqrt(1-abar_t),
@@ -34,21 +38,26 @@ struct DdimCoef {
 // Host: fill the coefficients from the SD scaled-linear schedule.
 void ddim_coefficients(DdimCoef* out);
 
-// Host launchers. frame_elems = latent_c * H * W (multiple of 4).
+// Host launchers. frame_elems = latent_c * H * W (multiple of 4). With
+// `sessions` > 1 every buffer (and the DevState array) carries a leading
+// session dimension: ring [S][16][fe], slot/batch motion [S][16][512], bank
+// [S][capacity][512], per-call inputs [S][...]; one grid slice per session.
 cudaError_t launch_prefill(DevState* st, float* ring, float* slot_motion, float* bank,
                            const float* ref_latent, const float* prefill_eps,
                            const float* ref_motion, const float* drive0, int64_t frame_elems,
-                           cudaStream_t s);
+                           int capacity, int sessions, cudaStream_t s);
 cudaError_t launch_ring_push(DevState* st, float* ring, float* slot_motion, float* batch_motion,
                              const float* new_noise, const float* new_motion,
-                             int64_t frame_elems, cudaStream_t s);
+                             int64_t frame_elems, int sessions, cudaStream_t s);
 cudaError_t launch_ddim(DevState* st, float* ring, const float* eps, float* out_x0,
-                        int64_t frame_elems, const DdimCoef& coef, cudaStream_t s);
-cudaError_t launch_ring_commit(DevState* st, cudaStream_t s);
+                        int64_t frame_elems, const DdimCoef& coef, int sessions, cudaStream_t s);
+cudaError_t launch_ring_commit(DevState* st, int sessions, cudaStream_t s);
+// With st != null the counts live in st[session] and `count`/`appends` are
+// ignored; without it (a standalone bank) sessions must be 1.
 cudaError_t launch_bank_check(float* bank, int32_t* count, int32_t* appends, int capacity,
                               int dim, const float* queries, int nq, double thr2, int cap,
                               int32_t* argmin, double* min_d2, uint8_t* appended,
-                              DevState* st, cudaStream_t s);
+                              DevState* st, int sessions, cudaStream_t s);
 // argmin_j ||query - store_j||^2 over `count` stored vectors (fp64, lowest index on ties).
 cudaError_t launch_nearest(const float* store, int count, int dim, const float* query,
                            int32_t* argmin, double* min_d2, cudaStream_t s);

@@ -20,6 +20,7 @@ using pl::GemmParams;
 namespace {
 
 constexpr size_t kAlign = 256;
+constexpr int kMaxSessions = 8;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
@@ -50,17 +51,18 @@ pl_status gemm_status(int r) {
 
 struct pl_ctx {
   pl_config cfg;
+  int sessions;        // S independent streams; per-stream buffers are [S][...]
   int capacity;        // motion/KV bank capacity = 1 + append_cap
   int64_t frame_elems; // latent_c * H * W
   uint8_t* ws;
   size_t ws_bytes;
-  pl::DevState* st;
+  pl::DevState* st;    // [S]
   float* ring;
   float* slot_motion;
   float* batch_motion;
   float* bank;
-  __half* bank_kv[PL_MAX_LAYERS];
-  float* motion_kv[PL_MAX_LAYERS];   // fp32 [16][32][2C]
+  __half* bank_kv[PL_MAX_LAYERS];     // fp16 [S][capacity][N][2C]
+  float* motion_kv[PL_MAX_LAYERS];   // fp32 [S][16][32][2C]
   __half* qkv;
   __half* attn_o;
   __half* a1;
@@ -91,22 +93,23 @@ size_t layout(const pl_config& c, pl_ctx* ctx) {
     return p;
   };
   const int capacity = 1 + c.append_cap;
+  const int64_t S = c.sessions > 0 ? c.sessions : 1;
   const int64_t fe = static_cast<int64_t>(c.latent_c) * c.latent_h * c.latent_w;
-  uint8_t* st = take(sizeof(pl::DevState));
-  uint8_t* ring = take(sizeof(float) * 16 * fe);
-  uint8_t* sm = take(sizeof(float) * 16 * 512);
-  uint8_t* bm = take(sizeof(float) * 16 * 512);
-  uint8_t* bank = take(sizeof(float) * capacity * 512);
+  uint8_t* st = take(sizeof(pl::DevState) * S);
+  uint8_t* ring = take(sizeof(float) * S * 16 * fe);
+  uint8_t* sm = take(sizeof(float) * S * 16 * 512);
+  uint8_t* bm = take(sizeof(float) * S * 16 * 512);
+  uint8_t* bank = take(sizeof(float) * S * capacity * 512);
   int64_t max_nc = 0;
   for (int l = 0; l < c.n_layers; ++l) {
     const int64_t N = c.layer_tokens[l], C = c.layer_channels[l];
-    uint8_t* bkv = take(sizeof(__half) * capacity * N * 2 * C);
-    uint8_t* mkv = take(sizeof(float) * 16 * 32 * 2 * C);
+    uint8_t* bkv = take(sizeof(__half) * S * capacity * N * 2 * C);
+    uint8_t* mkv = take(sizeof(float) * S * 16 * 32 * 2 * C);
     if (ctx) {
       ctx->bank_kv[l] = reinterpret_cast<__half*>(bkv);
       ctx->motion_kv[l] = reinterpret_cast<float*>(mkv);
     }
-    if (16 * N * C > max_nc) max_nc = 16 * N * C;
+    if (S * 16 * N * C > max_nc) max_nc = S * 16 * N * C;
   }
   uint8_t* qkv = take(sizeof(__half) * 3 * max_nc);
   uint8_t* ao = take(sizeof(__half) * max_nc);
@@ -138,6 +141,7 @@ pl_status validate_config(const pl_config* c) {
   if (c->heads < 1) return PL_EINVAL;
   if (c->append_cap < 0 || c->append_cap > PL_MAX_BANK - 1) return PL_EINVAL;
   if (!(c->drift_threshold >= 0.f) || !std::isfinite(c->drift_threshold)) return PL_EINVAL;
+  if (c->sessions < 0 || c->sessions > kMaxSessions) return PL_EINVAL;
   for (int l = 0; l < c->n_layers; ++l) {
     const int N = c->layer_tokens[l], C = c->layer_channels[l];
     if (N < 1 || C < 1 || C % c->heads || C % 16) return PL_EINVAL;
@@ -146,26 +150,36 @@ pl_status validate_config(const pl_config* c) {
   return PL_OK;
 }
 
-// Grouped K/V projection of bank features into entry `entry` of every layer.
-pl_status project_bank(pl_ctx* ctx, const void* const* feats, int entry, const int32_t* pred,
+// Grouped K/V projection of bank features (device fp16 [S][N_l][C_l] per
+// layer) into entry `entry` of every layer, one grouped launch per session;
+// with `predicated` a session's launch only runs when that session's bank
+// check appended anchor `entry` this round.
+pl_status project_bank(pl_ctx* ctx, const void* const* feats, int entry, bool predicated,
                        cudaStream_t s) {
-  GemmParams gp;
-  std::memset(&gp, 0, sizeof(gp));
-  gp.status = &ctx->st->status;
-  int np = 0;
-  for (int l = 0; l < ctx->cfg.n_layers; ++l) {
-    if (!feats[l]) return PL_EINVAL;
-    const int N = ctx->cfg.layer_tokens[l], C = ctx->cfg.layer_channels[l];
-    const __half* wkv = static_cast<const __half*>(ctx->w[l].w_qkv) + C;
-    __half* dst = ctx->bank_kv[l] + static_cast<int64_t>(entry) * N * 2 * C;
-    const int r = pl::gemm_make_problem(&gp.prob[np], feats[l], C, wkv, 3 * C, dst, 2 * C, N,
-                                        2 * C, C, pred);
-    if (r) return gemm_status(r);
-    ++np;
+  for (int z = 0; z < ctx->sessions; ++z) {
+    GemmParams gp;
+    std::memset(&gp, 0, sizeof(gp));
+    gp.status = &ctx->st[z].status;
+    const int32_t* pred = predicated ? &ctx->st[z].anchor_fire[entry] : nullptr;
+    int np = 0;
+    for (int l = 0; l < ctx->cfg.n_layers; ++l) {
+      if (!feats[l]) return PL_EINVAL;
+      const int64_t N = ctx->cfg.layer_tokens[l], C = ctx->cfg.layer_channels[l];
+      const __half* wkv = static_cast<const __half*>(ctx->w[l].w_qkv) + C;
+      const __half* a = static_cast<const __half*>(feats[l]) + z * N * C;
+      __half* dst = ctx->bank_kv[l] + (static_cast<int64_t>(z) * ctx->capacity + entry) * N * 2 * C;
+      const int r = pl::gemm_make_problem(&gp.prob[np], a, C, wkv, 3 * C, dst, 2 * C,
+                                          static_cast<int>(N), static_cast<int>(2 * C),
+                                          static_cast<int>(C), pred);
+      if (r) return gemm_status(r);
+      ++np;
+    }
+    gp.n_problems = np;
+    if (np == 0) return PL_OK;
+    const pl_status r = gemm_status(pl::gemm_launch(&gp, s, num_sms()));
+    if (r) return r;
   }
-  gp.n_problems = np;
-  if (np == 0) return PL_OK;
-  return gemm_status(pl::gemm_launch(&gp, s, num_sms()));
+  return PL_OK;
 }
 
 pl_status single_gemm(const void* a, int64_t lda, const void* b, int64_t ldb, void* c,
@@ -194,35 +208,45 @@ struct RoundArgs {
 // Enqueue one whole round on `s` (also used under stream capture).
 pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
   const pl_config& c = ctx->cfg;
+  const int S = ctx->sessions;
+  const int F = 16 * S;   // the batches of all sessions, session-major
   pl_status r = from_cuda(pl::launch_ring_push(ctx->st, ctx->ring, ctx->slot_motion,
                                                ctx->batch_motion, a.new_noise, a.new_motion,
-                                               ctx->frame_elems, s));
+                                               ctx->frame_elems, S, s));
   if (r) return r;
   for (int l = 0; l < c.n_layers; ++l) {
     const int N = c.layer_tokens[l], C = c.layer_channels[l], H = c.heads, hd = C / H;
-    const int64_t M = 16ll * N;
+    const int64_t M = static_cast<int64_t>(F) * N;
     const pl_layer_weights& w = ctx->w[l];
     __half* out = a.layer_out ? static_cast<__half*>(a.layer_out[l]) : ctx->out_default;
-    r = from_cuda(pl::launch_motion_kv(ctx->batch_motion, static_cast<const __half*>(w.m_kv), 16,
+    r = from_cuda(pl::launch_motion_kv(ctx->batch_motion, static_cast<const __half*>(w.m_kv), F,
                                        C, ctx->motion_kv[l], s));
     if (r) return r;
     r = single_gemm(a.hidden[l], C, w.w_qkv, 3 * C, ctx->qkv, 3 * C, static_cast<int>(M), 3 * C,
                     C, &ctx->st->status, s);
     if (r) return r;
+    // own K/V per frame; bank entry b of session z for the frames of session z
     AttnSegHost segs[1 + PL_MAX_BANK];
     segs[0] = {ctx->qkv + C, ctx->qkv + 2 * C, N, 3ll * C, static_cast<int64_t>(N) * 3 * C};
     const int nb = ctx->have_anchors ? ctx->capacity : 1;
     for (int b = 0; b < nb; ++b) {
       const __half* kv = ctx->bank_kv[l] + static_cast<int64_t>(b) * N * 2 * C;
       segs[1 + b] = {kv, kv + C, N, 2ll * C, 0};
+      if (S > 1) {
+        segs[1 + b].frame_stride = static_cast<int64_t>(ctx->capacity) * N * 2 * C;
+        segs[1 + b].n_blocks = S;
+        segs[1 + b].frame_div = 16;
+      }
     }
     AttnParams ap;
     int ar = pl::attn_make_params(&ap, ctx->qkv, 3ll * C, static_cast<int64_t>(N) * 3 * C, segs,
-                                  1 + nb, 16, N, H, hd, ctx->attn_o, C,
+                                  1 + nb, F, N, H, hd, ctx->attn_o, C,
                                   static_cast<int64_t>(N) * C);
     if (ar) return ar == 1 ? PL_EINVAL : PL_ECUDA;
     ap.n_fixed = 2;
     ap.n_extra = ctx->have_anchors ? &ctx->st->appends : nullptr;
+    ap.extra_div = 16;
+    ap.extra_stride = static_cast<int>(sizeof(pl::DevState) / sizeof(int32_t));
     ap.status = &ctx->st->status;
     ar = pl::attn_launch(ap, hd, s);
     if (ar) return ar == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
@@ -232,24 +256,24 @@ pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
     r = single_gemm(ctx->a1, C, w.m_q, C, ctx->qm, C, static_cast<int>(M), C, C,
                     &ctx->st->status, s, /*out_f32=*/true);
     if (r) return r;
-    r = from_cuda(pl::launch_motion_attn(ctx->qm, C, ctx->motion_kv[l], 16, N, C, H, ctx->om, C, s));
+    r = from_cuda(pl::launch_motion_attn(ctx->qm, C, ctx->motion_kv[l], F, N, C, H, ctx->om, C, s));
     if (r) return r;
     r = single_gemm(ctx->om, C, w.m_o, C, out, C, static_cast<int>(M), C, C, &ctx->st->status, s);
     if (r) return r;
   }
   r = from_cuda(pl::launch_ddim(ctx->st, ctx->ring, a.eps, a.out_frames, ctx->frame_elems,
-                                ctx->coef, s));
+                                ctx->coef, S, s));
   if (r) return r;
-  r = from_cuda(pl::launch_ring_commit(ctx->st, s));
+  r = from_cuda(pl::launch_ring_commit(ctx->st, S, s));
   if (r) return r;
-  r = from_cuda(pl::launch_bank_check(ctx->bank, &ctx->st->bank_count, &ctx->st->appends,
-                                      ctx->capacity, 512, a.new_motion, 4,
+  r = from_cuda(pl::launch_bank_check(ctx->bank, nullptr, nullptr, ctx->capacity, 512,
+                                      a.new_motion, 4,
                                       static_cast<double>(c.drift_threshold) * c.drift_threshold,
-                                      c.append_cap, nullptr, nullptr, a.appended, ctx->st, s));
+                                      c.append_cap, nullptr, nullptr, a.appended, ctx->st, S, s));
   if (r) return r;
   if (ctx->have_anchors) {
     for (int an = 1; an <= c.append_cap; ++an) {
-      r = project_bank(ctx, ctx->anchor_feats[an - 1], an, &ctx->st->anchor_fire[an], s);
+      r = project_bank(ctx, ctx->anchor_feats[an - 1], an, /*predicated=*/true, s);
       if (r) return r;
     }
   }
@@ -458,7 +482,7 @@ pl_status pl_motion_bank_check(float* bank, int32_t* count, int32_t* appends, in
   if (n_queries == 0) return PL_OK;
   const double thr2 = static_cast<double>(threshold) * threshold;
   return from_cuda(pl::launch_bank_check(bank, count, appends, capacity, dim, queries, n_queries,
-                                         thr2, cap, argmin, min_d2, appended, nullptr,
+                                         thr2, cap, argmin, min_d2, appended, nullptr, 1,
                                          static_cast<cudaStream_t>(stream)));
 }
 
@@ -508,6 +532,7 @@ pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_
   if (!ctx) return PL_ENOMEM;
   std::memset(static_cast<void*>(ctx), 0, sizeof(*ctx));
   ctx->cfg = *cfg;
+  ctx->sessions = cfg->sessions > 0 ? cfg->sessions : 1;
   ctx->capacity = 1 + cfg->append_cap;
   ctx->frame_elems = static_cast<int64_t>(cfg->latent_c) * cfg->latent_h * cfg->latent_w;
   ctx->ws = static_cast<uint8_t*>(workspace);
@@ -521,7 +546,7 @@ pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_
     return PL_ECUDA;
   }
   // zero the device state so pl_get_state is meaningful before bank_init
-  if (cudaMemset(ctx->st, 0, sizeof(pl::DevState)) != cudaSuccess) {
+  if (cudaMemset(ctx->st, 0, sizeof(pl::DevState) * ctx->sessions) != cudaSuccess) {
     delete ctx;
     return PL_ECUDA;
   }
@@ -561,10 +586,10 @@ pl_status pl_bank_init(pl_ctx* ctx, const pl_layer_weights* weights,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   pl_status r = from_cuda(pl::launch_prefill(ctx->st, ctx->ring, ctx->slot_motion, ctx->bank,
                                              ref_latent, prefill_eps, ref_motion, drive0_motion,
-                                             ctx->frame_elems, s));
+                                             ctx->frame_elems, ctx->capacity, ctx->sessions, s));
   if (r) return r;
   if (L > 0) {
-    r = project_bank(ctx, ctx->ref_feats, 0, nullptr, s);
+    r = project_bank(ctx, ctx->ref_feats, 0, /*predicated=*/false, s);
     if (r) return r;
   }
   ctx->initialised = true;
@@ -576,7 +601,7 @@ pl_status pl_ring_push(pl_ctx* ctx, const float* new_noise, const float* new_mot
   if (!ctx || !new_noise || !new_motion) return PL_EINVAL;
   if (!ctx->initialised) return PL_ESTATE;
   return from_cuda(pl::launch_ring_push(ctx->st, ctx->ring, ctx->slot_motion, ctx->batch_motion,
-                                        new_noise, new_motion, ctx->frame_elems,
+                                        new_noise, new_motion, ctx->frame_elems, ctx->sessions,
                                         static_cast<cudaStream_t>(stream)));
 }
 
@@ -586,9 +611,9 @@ pl_status pl_pyramid_ddim_step(pl_ctx* ctx, const float* eps, float* out_x0, voi
   if (!aligned16(eps) || !aligned16(out_x0)) return PL_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   pl_status r = from_cuda(pl::launch_ddim(ctx->st, ctx->ring, eps, out_x0, ctx->frame_elems,
-                                          ctx->coef, s));
+                                          ctx->coef, ctx->sessions, s));
   if (r) return r;
-  return from_cuda(pl::launch_ring_commit(ctx->st, s));
+  return from_cuda(pl::launch_ring_commit(ctx->st, ctx->sessions, s));
 }
 
 pl_status pl_ctx_bank_check(pl_ctx* ctx, const float* queries, int n_queries, int32_t* argmin,
@@ -599,13 +624,13 @@ pl_status pl_ctx_bank_check(pl_ctx* ctx, const float* queries, int n_queries, in
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const pl_config& c = ctx->cfg;
   pl_status r = from_cuda(pl::launch_bank_check(
-      ctx->bank, &ctx->st->bank_count, &ctx->st->appends, ctx->capacity, 512, queries, n_queries,
+      ctx->bank, nullptr, nullptr, ctx->capacity, 512, queries, n_queries,
       static_cast<double>(c.drift_threshold) * c.drift_threshold, c.append_cap, argmin, min_d2,
-      appended, ctx->st, s));
+      appended, ctx->st, ctx->sessions, s));
   if (r) return r;
   if (ctx->have_anchors) {
     for (int an = 1; an <= c.append_cap; ++an) {
-      r = project_bank(ctx, ctx->anchor_feats[an - 1], an, &ctx->st->anchor_fire[an], s);
+      r = project_bank(ctx, ctx->anchor_feats[an - 1], an, /*predicated=*/true, s);
       if (r) return r;
     }
   }
@@ -668,12 +693,13 @@ pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_
   return from_cuda(cudaGraphLaunch(ctx->exec, s));
 }
 
-pl_status pl_get_state(pl_ctx* ctx, pl_state* out, void* stream) {
-  if (!ctx || !out) return PL_EINVAL;
+pl_status pl_get_session_state(pl_ctx* ctx, int session, pl_state* out, void* stream) {
+  if (!ctx || !out || session < 0 || session >= ctx->sessions) return PL_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return PL_ECUDA;
   pl::DevState d;
-  if (cudaMemcpy(&d, ctx->st, sizeof(d), cudaMemcpyDeviceToHost) != cudaSuccess) return PL_ECUDA;
+  if (cudaMemcpy(&d, ctx->st + session, sizeof(d), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return PL_ECUDA;
   std::memset(out, 0, sizeof(*out));
   out->initialised = ctx->initialised ? d.initialised : 0;
   out->head = d.head;
@@ -687,19 +713,30 @@ pl_status pl_get_state(pl_ctx* ctx, pl_state* out, void* stream) {
   return PL_OK;
 }
 
-pl_status pl_get_motion_bank(pl_ctx* ctx, float* host_out, int32_t* count, void* stream) {
-  if (!ctx || !host_out || !count) return PL_EINVAL;
+pl_status pl_get_state(pl_ctx* ctx, pl_state* out, void* stream) {
+  return pl_get_session_state(ctx, 0, out, stream);
+}
+
+pl_status pl_get_session_motion_bank(pl_ctx* ctx, int session, float* host_out, int32_t* count,
+                                     void* stream) {
+  if (!ctx || !host_out || !count || session < 0 || session >= ctx->sessions) return PL_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return PL_ECUDA;
   int32_t n = 0;
-  if (cudaMemcpy(&n, &ctx->st->bank_count, sizeof(n), cudaMemcpyDeviceToHost) != cudaSuccess)
+  if (cudaMemcpy(&n, &ctx->st[session].bank_count, sizeof(n), cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
     return PL_ECUDA;
   if (n < 0 || n > ctx->capacity) return PL_EDEVICE;
   *count = n;
-  if (n > 0 && cudaMemcpy(host_out, ctx->bank, sizeof(float) * 512 * n, cudaMemcpyDeviceToHost) !=
-                   cudaSuccess)
+  const float* bank = ctx->bank + static_cast<int64_t>(session) * ctx->capacity * 512;
+  if (n > 0 &&
+      cudaMemcpy(host_out, bank, sizeof(float) * 512 * n, cudaMemcpyDeviceToHost) != cudaSuccess)
     return PL_ECUDA;
   return PL_OK;
+}
+
+pl_status pl_get_motion_bank(pl_ctx* ctx, float* host_out, int32_t* count, void* stream) {
+  return pl_get_session_motion_bank(ctx, 0, host_out, count, stream);
 }
 
 pl_status pl_get_device_status(pl_ctx* ctx, void* stream) {
@@ -707,11 +744,16 @@ pl_status pl_get_device_status(pl_ctx* ctx, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return PL_ECUDA;
   uint32_t w = 0;
-  if (cudaMemcpy(&w, &ctx->st->status, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess)
-    return PL_ECUDA;
-  const uint32_t zero = 0;
-  if (cudaMemcpy(&ctx->st->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
-    return PL_ECUDA;
+  for (int z = 0; z < ctx->sessions; ++z) {
+    uint32_t wz = 0;
+    if (cudaMemcpy(&wz, &ctx->st[z].status, sizeof(wz), cudaMemcpyDeviceToHost) != cudaSuccess)
+      return PL_ECUDA;
+    const uint32_t zero = 0;
+    if (cudaMemcpy(&ctx->st[z].status, &zero, sizeof(zero), cudaMemcpyHostToDevice) !=
+        cudaSuccess)
+      return PL_ECUDA;
+    w |= wz;
+  }
   if (w & pl::DEV_TIMEOUT) return PL_ETIMEOUT;
   if (w) return PL_EDEVICE;
   return PL_OK;

@@ -235,7 +235,16 @@ typedef struct pl_config {
   int32_t heads;                         /* 8 */
   float drift_threshold;                 /* 17 */
   int32_t append_cap;                    /* 3 (so the bank holds at most 4) */
+  int32_t sessions;                      /* independent streams served together, 1..8
+                                            (0 is read as 1); see below */
 } pl_config;
+
+/* Sessions. A context serves S = cfg.sessions independent streams (same
+ * weights, separate piles, banks and states) in the same launches: one
+ * round of every session is one pl_stream_round. Every per-stream buffer
+ * argument of the calls below then carries a leading session dimension
+ * [S] in front of the shape given (session s at offset s times the
+ * per-session size); for S = 1 the shapes are exactly as written. */
 
 /* Per-layer weights (device fp16, row-major [in][out]); kept by pointer, so
  * they must outlive the context. */
@@ -323,18 +332,26 @@ pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_
                           const void* const* hidden, const float* eps, float* out_frames,
                           uint8_t* appended, void* const* layer_out, void* stream);
 
-/* Synchronise `stream` and copy the context's state to *out. */
+/* Synchronise `stream` and copy the state of session 0 to *out. */
 pl_status pl_get_state(pl_ctx* ctx, pl_state* out, void* stream);
 
-/* Synchronise `stream`, copy the motion bank (fp32 [count][512]) to host. */
+/* The same for session `session` (0 <= session < S). */
+pl_status pl_get_session_state(pl_ctx* ctx, int session, pl_state* out, void* stream);
+
+/* Synchronise `stream`, copy the motion bank (fp32 [count][512]) of session
+ * 0 to host. */
 pl_status pl_get_motion_bank(pl_ctx* ctx, float* host_out, int32_t* count, void* stream);
 
-/* Synchronise `stream` and map the device status word to a status:
- * PL_OK, PL_ETIMEOUT or PL_EDEVICE. Clears the word. */
+/* The same for session `session`. */
+pl_status pl_get_session_motion_bank(pl_ctx* ctx, int session, float* host_out, int32_t* count,
+                                     void* stream);
+
+/* Synchronise `stream` and map the device status words of all sessions to a
+ * status: PL_OK, PL_ETIMEOUT or PL_EDEVICE. Clears the words. */
 pl_status pl_get_device_status(pl_ctx* ctx, void* stream);
 
-/* Device pointer of the pile's latents, fp32 [4 slots][4][4][H][W] (read-only
- * view for tests; slot s holds the window at timestep slot_t[s]). */
+/* Device pointer of the piles' latents, fp32 [S][4 slots][4][4][H][W]
+ * (read-only view for tests; slot s holds the window at timestep slot_t[s]). */
 const float* pl_ctx_ring_latents(const pl_ctx* ctx);
 
 #ifdef __cplusplus

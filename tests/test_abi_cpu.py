@@ -73,6 +73,25 @@ def test_config_validation_and_workspace_size():
     assert P.lib.pl_ctx_create(C.byref(cfg), C.c_void_p(256), 16, C.byref(h)) == P.PL_ENOMEM
 
 
+def test_sessions_scale_the_workspace():
+    import denoise_step_b200 as P
+    import synthetic as S
+    layers = [(side * side, c) for _, side, c in S.LAYERS]
+    n = C.c_size_t()
+    sizes = {}
+    for sess in (0, 1, 2, 4, 8):
+        cfg = P.make_config((64, 64), layers, sessions=sess)
+        assert P.lib.pl_workspace_bytes(C.byref(cfg), C.byref(n)) == P.PL_OK
+        sizes[sess] = n.value
+    assert sizes[0] == sizes[1]                        # 0 is read as one session
+    # every buffer is per session (256-byte rounding aside)
+    assert abs(sizes[2] - 2 * sizes[1]) < 64 * 256
+    assert abs(sizes[8] - 8 * sizes[1]) < 256 * 256
+    for sess in (-1, 9):
+        cfg = P.make_config((64, 64), layers, sessions=sess)
+        assert P.lib.pl_workspace_bytes(C.byref(cfg), C.byref(n)) == P.PL_EINVAL
+
+
 def test_round_before_init_is_a_state_error():
     import denoise_step_b200 as P
     # a null context is rejected before any device work
