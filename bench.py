@@ -317,6 +317,39 @@ def sessions_round(torch, P, wl, stream, sessions, single_ms):
             "frames_per_s": 4 * sessions / t, "speedup_vs_one_session": sessions * single_ms / (t * 1e3)}
 
 
+def sink_stream_step(torch, P, stream):
+    """PR-Sink cache at the C5 sizes (4096 tokens x 40 heads x 128, pool of 64
+    pose-descriptor blocks of 64-d): steps with the cache full (own + sink + 3
+    rolling + 1 retrieved = 6 x 4096 keys), each timed by CUDA events around
+    pl_sink_step alone (the caller's K/V writes stay outside)."""
+    n, heads, hd, pool, dim = 4096, 40, 128, 64, 64
+    g = torch.Generator(device="cuda").manual_seed(SEED)
+    sink = P.Sink(n, heads, hd, pool, dim)
+    q = torch.randn((n, heads * hd), device="cuda", dtype=torch.float16, generator=g)
+    kv = torch.randn((2, n, heads * hd), device="cuda", dtype=torch.float16, generator=g)
+    poses = torch.randn((16, dim), device="cuda", generator=g)
+    out = torch.empty_like(q)
+    times = []
+    with torch.cuda.stream(stream):
+        for t in range(12):
+            kd, vd = sink.block_kv()
+            kd.copy_(kv[0])
+            vd.copy_(kv[1])
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            sink.step(q, poses[t], out=out, stream=stream)
+            e1.record(stream)
+            times.append((e0, e1))
+    stream.synchronize()
+    st = sink.state(stream)
+    sink.close()
+    steady = [a.elapsed_time(b) for a, b in times[6:]]     # pool non-empty from step 5
+    ms = sum(steady) / len(steady)
+    fl = 4.0 * n * 6 * n * hd * heads
+    return {"ms_per_step": ms, "tflops": fl / ms / 1e9, "steps_timed": len(steady),
+            "pool_count": st["pool_count"], "n_roll": st["n_roll"]}
+
+
 def secondary_measurements(torch, P, stream, hbm_peak):
     """The other workloads' kernels, timed live (CUDA events on their stream):
     the PR-Sink block (4096 tokens x 40 heads x 128, KV own + sink + retrieved
@@ -497,6 +530,7 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and not args.no_secondary:
         sec = secondary_measurements(torch, P, stream, hbm_peak)
         sec["sessions_4"] = sessions_round(torch, P, wl, stream, 4, elapsed / args.steps * 1e3)
+        sec["pr_sink_cache_step"] = sink_stream_step(torch, P, stream)
         line["config"]["secondary"] = sec
     clk = clocks_summary(clk_path)
     if clk is not None:

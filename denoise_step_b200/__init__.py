@@ -43,6 +43,15 @@ class Config(C.Structure):
                 ("sessions", C.c_int32)]
 
 
+class SinkState(C.Structure):
+    _fields_ = [("blocks", C.c_int64), ("has_sink", C.c_int32), ("n_roll", C.c_int32),
+                ("pool_count", C.c_int32), ("retrieved", C.c_int32), ("retrieved_d2", C.c_double),
+                ("device_status", C.c_uint32)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
 class LayerWeights(C.Structure):
     _fields_ = [("w_qkv", vp), ("w_o", vp), ("m_q", vp), ("m_kv", vp), ("m_o", vp)]
 
@@ -90,6 +99,12 @@ _SIGS = {
     "pl_get_session_motion_bank": (i32, [vp, i32, vp, C.POINTER(C.c_int32), vp]),
     "pl_get_device_status": (i32, [vp, vp]),
     "pl_ctx_ring_latents": (vp, [vp]),
+    "pl_sink_workspace_bytes": (i32, [i32, i32, i32, i32, i32, C.POINTER(sz)]),
+    "pl_sink_create": (i32, [i32, i32, i32, i32, i32, vp, sz, C.POINTER(vp)]),
+    "pl_sink_destroy": (i32, [vp]),
+    "pl_sink_block_kv": (i32, [vp, C.POINTER(vp), C.POINTER(vp)]),
+    "pl_sink_step": (i32, [vp, vp, vp, vp, vp]),
+    "pl_sink_get_state": (i32, [vp, C.POINTER(SinkState), vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -367,3 +382,60 @@ class Stream:
 
     def ring_latents(self):
         return lib.pl_ctx_ring_latents(self.handle)
+
+
+class _DeviceArray:
+    """A device buffer the library owns, shown to torch without a copy."""
+
+    def __init__(self, ptr, shape, typestr):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 3}
+
+
+class Sink:
+    """PR-Sink bounded KV cache of one block stream (pl_sink_*)."""
+
+    def __init__(self, n, heads, head_dim, pool_capacity, pose_dim, device="cuda"):
+        import torch
+        self.n, self.heads, self.head_dim = n, heads, head_dim
+        need = sz()
+        check(lib.pl_sink_workspace_bytes(n, heads, head_dim, pool_capacity, pose_dim,
+                                          C.byref(need)), "pl_sink_workspace_bytes")
+        self.workspace = torch.empty(need.value, dtype=torch.uint8, device=device)
+        h = vp()
+        check(lib.pl_sink_create(n, heads, head_dim, pool_capacity, pose_dim,
+                                 _ptr(self.workspace), need.value, C.byref(h)), "pl_sink_create")
+        self.handle = h
+
+    def close(self):
+        if self.handle:
+            lib.pl_sink_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def block_kv(self):
+        """torch views [n, heads*head_dim] fp16 of where the next block's K and V go."""
+        import torch
+        k, v = vp(), vp()
+        check(lib.pl_sink_block_kv(self.handle, C.byref(k), C.byref(v)), "pl_sink_block_kv")
+        shape = (self.n, self.heads * self.head_dim)
+        return (torch.as_tensor(_DeviceArray(k.value, shape, "<f2"), device="cuda"),
+                torch.as_tensor(_DeviceArray(v.value, shape, "<f2"), device="cuda"))
+
+    def step(self, q, pose, out=None, stream=None):
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        check(lib.pl_sink_step(self.handle, _ptr(_contig(q, "q")), _ptr(pose), _ptr(out),
+                               _stream(stream)), "pl_sink_step")
+        return out
+
+    def state(self, stream=None):
+        s = SinkState()
+        check(lib.pl_sink_get_state(self.handle, C.byref(s), _stream(stream)), "pl_sink_get_state")
+        return s.as_dict()

@@ -214,6 +214,57 @@ pl_status pl_nearest(const float* store, int64_t count, int dim, const float* qu
                      void* stream);
 
 /* ------------------------------------------------------------------ *
+ * PR-Sink cache: the bounded KV cache of one block-streaming generator
+ * ------------------------------------------------------------------ */
+
+/* LiveAnimate page, PR-Sink: a bounded KV cache in three parts, the static
+ * sink (the first generated block, kept for good), one dynamic block chosen
+ * by pose from the history, and a rolling buffer of three slots; memory and
+ * per-block cost stay constant however long the stream runs. Readings of
+ * what the page leaves open: a block enters the rolling buffer after its own
+ * step (the first block becomes the sink instead); the block a full rolling
+ * buffer pushes out enters the pose pool with its pose descriptor; a full
+ * pool replaces its oldest entry; the dynamic block is the pool entry
+ * nearest to the current block's pose (squared L2 in fp64, lowest pool slot
+ * on equal distances), attended only while the pool is not empty.
+ *
+ * One step: out = softmax(q K_cat^T / sqrt(head_dim)) V_cat over
+ *   K_cat = [own ; sink ; rolling (oldest first) ; pool[j*]]   (V alike),
+ * each part present once it exists; then the cache update above. Blocks
+ * live in a device arena of pool_capacity + 5 blocks inside the caller's
+ * workspace and never move: the sink, the rolling buffer and the pool are
+ * index lists, so a step copies no K/V. The caller writes the current
+ * block's K and V (fp16 [n][heads*head_dim]) at the pointers
+ * pl_sink_block_kv returns, before pl_sink_step. */
+typedef struct pl_sink pl_sink;
+
+typedef struct pl_sink_state {
+  int64_t blocks;         /* steps taken */
+  int32_t has_sink;
+  int32_t n_roll;         /* blocks in the rolling buffer (0..3) */
+  int32_t pool_count;     /* entries in the pose pool */
+  int32_t retrieved;      /* pool slot attended by the last step, -1 when none */
+  double retrieved_d2;    /* its squared pose distance (0 when none) */
+  uint32_t device_status;
+} pl_sink_state;
+
+pl_status pl_sink_workspace_bytes(int n, int heads, int head_dim, int pool_capacity,
+                                  int pose_dim, size_t* bytes);
+/* n tokens per block (>= 1), head_dim in {40, 64, 80, 128, 160},
+ * 1 <= pool_capacity <= 4096, 1 <= pose_dim <= 4096; workspace: device,
+ * 256-byte aligned, >= pl_sink_workspace_bytes. */
+pl_status pl_sink_create(int n, int heads, int head_dim, int pool_capacity, int pose_dim,
+                         void* workspace, size_t workspace_bytes, pl_sink** out);
+pl_status pl_sink_destroy(pl_sink* sink);
+/* Device pointers where the next block's K and V go (fp16 [n][heads*head_dim]). */
+pl_status pl_sink_block_kv(pl_sink* sink, void** k, void** v);
+/* One block: q, out device fp16 [n][heads*head_dim]; pose: device fp32
+ * [pose_dim], the block's pose descriptor. */
+pl_status pl_sink_step(pl_sink* sink, const void* q, const float* pose, void* out, void* stream);
+/* Synchronise `stream` and report the cache state. */
+pl_status pl_sink_get_state(pl_sink* sink, pl_sink_state* out, void* stream);
+
+/* ------------------------------------------------------------------ *
  * Stream context: the device-resident pile and the reference bank
  * ------------------------------------------------------------------ */
 

@@ -247,6 +247,65 @@ def pose_retrieve(store: np.ndarray, desc: np.ndarray) -> int:
     return int(np.argmin(d2))
 
 
+class PRSinkCache:
+    """[LA] PR-Sink: the bounded KV cache of one block stream.
+
+    Parts (the page): the static sink (the first generated block, kept for
+    good), one dynamic block retrieved from the history by pose, and a
+    rolling buffer of three blocks. Readings where the page is silent: a
+    block joins the cache after its own step (the first one as the sink, the
+    others in the rolling buffer); the block a full rolling buffer pushes out
+    enters the pose pool with its descriptor; a full pool replaces its oldest
+    entry; retrieval is pose_retrieve over the pool in slot order and only
+    happens once the pool holds something. Attention of a block: full
+    (non-causal) over [own ; sink ; rolling oldest first ; retrieved].
+    """
+
+    ROLLING = 3
+
+    def __init__(self, pool_capacity: int, heads: int):
+        self.pool_capacity, self.heads = pool_capacity, heads
+        self.sink = None            # (k, v)
+        self.rolling = deque()      # (k, v, pose), oldest first
+        self.pool = []              # (k, v, pose) per pool slot
+        self.pool_oldest = 0        # slot a full pool replaces next
+        self.blocks = 0
+
+    def parts(self, pose):
+        """The cache's K/V parts a block with this pose attends, and the retrieved slot."""
+        ks, vs = [], []
+        if self.sink is not None:
+            ks.append(self.sink[0])
+            vs.append(self.sink[1])
+        for k, v, _ in self.rolling:
+            ks.append(k)
+            vs.append(v)
+        slot = None
+        if self.pool:
+            slot = pose_retrieve(np.array([p for _, _, p in self.pool]), pose)
+            ks.append(self.pool[slot][0])
+            vs.append(self.pool[slot][1])
+        return ks, vs, slot
+
+    def step(self, q, k, v, pose):
+        """Attention of block q (own K/V k, v) over the cache, then the cache update."""
+        ks, vs, slot = self.parts(pose)
+        out = segment_attention(q, [k] + ks, [v] + vs, self.heads)
+        if self.sink is None:
+            self.sink = (k, v)
+        else:
+            if len(self.rolling) == self.ROLLING:
+                old = self.rolling.popleft()
+                if len(self.pool) < self.pool_capacity:
+                    self.pool.append(old)
+                else:
+                    self.pool[self.pool_oldest] = old
+                    self.pool_oldest = (self.pool_oldest + 1) % self.pool_capacity
+            self.rolling.append((k, v, np.asarray(pose)))
+        self.blocks += 1
+        return out, slot
+
+
 # ---------------------------------------------------------------------------
 # Prefill. [PL] "首帧怎么办".
 # ---------------------------------------------------------------------------

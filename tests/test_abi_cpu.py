@@ -97,3 +97,20 @@ def test_round_before_init_is_a_state_error():
     # a null context is rejected before any device work
     assert P.lib.pl_stream_round(None, None, None, None, None, None, None, None, None) == P.PL_EINVAL
     assert P.lib.pl_ring_push(None, None, None, None) == P.PL_EINVAL
+
+
+def test_sink_validation():
+    import denoise_step_b200 as P
+    n = C.c_size_t()
+    L = P.lib
+    assert L.pl_sink_workspace_bytes(4096, 40, 128, 64, 64, C.byref(n)) == P.PL_OK
+    # arena: pool + 5 blocks of K and V, each n * heads * head_dim fp16
+    assert n.value >= 2 * 69 * 4096 * 5120 * 2
+    assert L.pl_sink_workspace_bytes(4096, 40, 96, 64, 64, C.byref(n)) == P.PL_EUNSUPPORTED
+    assert L.pl_sink_workspace_bytes(4096, 40, 128, 0, 64, C.byref(n)) == P.PL_EINVAL
+    assert L.pl_sink_workspace_bytes(0, 40, 128, 64, 64, C.byref(n)) == P.PL_EINVAL
+    assert L.pl_sink_workspace_bytes(64, 1, 64, 4097, 8, C.byref(n)) == P.PL_EINVAL
+    h = C.c_void_p()
+    assert L.pl_sink_create(64, 1, 64, 2, 8, None, 0, C.byref(h)) == P.PL_EINVAL
+    assert L.pl_sink_create(64, 1, 64, 2, 8, C.c_void_p(256), 16, C.byref(h)) == P.PL_ENOMEM
+    assert L.pl_sink_step(None, None, None, None, None) == P.PL_EINVAL

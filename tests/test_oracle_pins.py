@@ -388,3 +388,64 @@ def test_motion_xattn_brute_force():
     m = S.normal(24, "m", (32, 16))
     want = _brute_attention((x @ w["mq"]).tolist(), (m @ w["mk"]).tolist(), (m @ w["mv"]).tolist(), 8) @ w["mo"]
     assert np.max(np.abs(O.motion_xattn_frame(x, m, w, 8) - want)) < 1e-12
+
+
+# ------------------------------------------------------------------ PR-Sink cache ([LA])
+
+def _block_kv(b, n=4, C=8):
+    """Block b: every key the same (so attention weights are uniform over the
+    attended tokens) and every value equal to b."""
+    return np.ones((n, C)), np.full((n, C), float(b))
+
+
+def test_pr_sink_cache_lifecycle():
+    # pool of 2: the hand-derived contents after each block (ids of the blocks)
+    cache = O.PRSinkCache(pool_capacity=2, heads=2)
+    want = {  # t: (rolling oldest first, pool by slot)
+        0: ([], []), 1: ([1], []), 2: ([1, 2], []), 3: ([1, 2, 3], []),
+        4: ([2, 3, 4], [1]), 5: ([3, 4, 5], [1, 2]), 6: ([4, 5, 6], [3, 2]),
+        7: ([5, 6, 7], [3, 4]),
+    }
+    for t in range(8):
+        k, v = _block_kv(t)
+        cache.step(np.ones((4, 8)), k, v, np.array([float(t)]))
+        roll, pool = want[t]
+        assert cache.sink[1][0, 0] == 0.0
+        assert [int(r[1][0, 0]) for r in cache.rolling] == roll
+        assert [int(p[1][0, 0]) for p in cache.pool] == pool
+        assert cache.blocks == t + 1
+
+
+def test_pr_sink_step_attends_own_sink_rolling_and_retrieved():
+    # with uniform weights the output is the mean of the attended blocks' values
+    cache = O.PRSinkCache(pool_capacity=2, heads=2)
+    means = []
+    for t in range(8):
+        k, v = _block_kv(t)
+        out, slot = cache.step(np.ones((4, 8)), k, v, np.array([float(t)]))
+        means.append(float(out[0, 0]))
+        # the pool first receives a block in the update of t = 4
+        assert (slot is None) == (t <= 4)
+    # t = 5: own 5, sink 0, rolling 2 3 4, pool {1} -> retrieved 1: mean 15 / 6
+    assert abs(means[5] - 15 / 6) < 1e-12
+    # t = 6: own 6, sink 0, rolling 3 4 5, pool {1, 2}, pose 6 nearest to 2's: (6+0+12+2)/6
+    assert abs(means[6] - 20 / 6) < 1e-12
+    # t = 1: own 1 + sink 0 only
+    assert abs(means[1] - 0.5) < 1e-12
+    assert abs(means[0] - 0.0) < 1e-12
+
+
+def test_pr_sink_retrieval_nearest_pose_lowest_slot_on_ties():
+    cache = O.PRSinkCache(pool_capacity=4, heads=1)
+    poses = [np.array([0.0, 0.0]), np.array([5.0, 0.0]), np.array([1.0, 0.0]),
+             np.array([-1.0, 0.0]), np.array([3.0, 3.0]), np.array([9.0, 9.0]),
+             np.array([9.0, 8.0])]
+    for t, ps in enumerate(poses):
+        k, v = _block_kv(t)
+        cache.step(np.ones((4, 8)), k, v, ps)
+    # pool holds blocks 1, 2, 3 (poses (5,0), (1,0), (-1,0)) in slots 0, 1, 2
+    assert [int(p[1][0, 0]) for p in cache.pool] == [1, 2, 3]
+    _, _, slot = cache.parts(np.array([0.0, 0.0]))    # (1,0) and (-1,0) tie
+    assert slot == 1
+    _, _, slot = cache.parts(np.array([4.0, 0.0]))
+    assert slot == 0
