@@ -25,14 +25,14 @@
 // The softmax is issue- and MUFU-bound (one exp2 per score at head_dim 40
 // against 160 tensor FLOPs), so its inner loop uses packed f32x2 FMAs,
 // 3-input max and one of two exp2 paths (EXPM): 0 = ex2.approx.f32 on the
-// MUFU pipe; 2 = MUFU for 3 of every 4 pairs and a degree-3 polynomial
-// on the FMA pipe for the 4th (Cody-Waite split 2^x = 2^n 2^f with n the
-// nearest integer, f in [-0.5, 0.5]; the cubic is fitted to 2^f on that
-// interval, max relative error 7.7e-5).
+// MUFU pipe; 2 = MUFU for most pairs and a degree-3 polynomial on the FMA
+// pipe for the pairs kPolyPairs marks (Cody-Waite split 2^x = 2^n 2^f with n
+// the nearest integer, f in [-0.5, 0.5]; the cubic is fitted to 2^f on that
+// interval, max relative error 7.7e-5, below the fp16 rounding of P).
 // Measured on B200 (level-64 kernel): ex2.approx.f32 issues 16 results per
 // clock per SM and ex2.approx.f16x2 only 8 instructions (the same 16 results),
-// so the f16x2 path was dropped; the polynomial split (EXPM 2) was 7% slower
-// than MUFU alone at this shape and is kept only as a compile-time option.
+// so the f16x2 path was dropped. With one MMA issuer the polynomial split was
+// slower (the tensor pipe set the pace); with two it takes 8% off head_dim 40.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -77,6 +77,8 @@ struct Cfg {
 };
 
 constexpr int kThreads = 384;
+// EXPM 2: bit e set = pair e of each 32-column chunk takes the FMA-pipe exp2
+constexpr uint32_t kPolyPairs = 0x9248u;
 constexpr int kRegsLaunch = 168;      // 384 x 168 >= 128 x 120 + 256 x 184
 constexpr int kRegsProducer = 120;
 constexpr int kRegsSoftmax = 184;
@@ -418,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             for (int e = 0; e < 16; ++e) {
               const uint64_t x = f2_fma(f2_pack(s[c + 2 * e], s[c + 2 * e + 1]), sc2, nm2);
               uint64_t pp;
-              if (EXPM == 2 && (e & 3) == 3) {
+              if (EXPM == 2 && ((kPolyPairs >> e) & 1)) {
                 pp = exp2_poly2(x);
               } else {
                 float x0, x1;
@@ -491,7 +493,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 // issuer at head_dim 160.
 template <int HD>
 constexpr int kVar = (HD <= 64) ? 2 : (HD <= 128 ? 1 : 0);
-constexpr int kExpMode = 0;   // exp2 on the MUFU pipe only
+// exp2 path per head dimension: at head_dim <= 64 the MUFU is the limit and
+// 5 of every 16 pairs go to the FMA-pipe polynomial (level-64 launch 3.39 ->
+// 3.12 ms; 4/16: 3.20, 6/16: 3.28, 2/16: 3.36 ms); at larger head dims the
+// tensor pipe leads and the polynomial measured slower (32x32 layer 0.307 ->
+// 0.317 ms, PR-Sink block 1.91 -> 2.00 ms), so MUFU only there.
+template <int HD>
+constexpr int kExpMode = (HD <= 64) ? 2 : 0;
 
 int block_n(int head_dim) {
   switch (head_dim) {
@@ -509,9 +517,9 @@ int set_attr() {
   constexpr int V = kVar<HD>;
   // the setmaxnreg split needs exactly kRegsLaunch registers per thread at launch
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, attn_kernel<HD, kExpMode, V>) != cudaSuccess) return 4;
+  if (cudaFuncGetAttributes(&fa, attn_kernel<HD, kExpMode<HD>, V>) != cudaSuccess) return 4;
   if (fa.numRegs != kRegsLaunch) return 4;
-  return cudaFuncSetAttribute(attn_kernel<HD, kExpMode, V>,
+  return cudaFuncSetAttribute(attn_kernel<HD, kExpMode<HD>, V>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(Cfg<HD, V>::SMEM)) == cudaSuccess ? 0 : 4;
 }
@@ -520,7 +528,7 @@ template <int HD>
 int launch_hd(const AttnParams& p, cudaStream_t stream) {
   constexpr int V = kVar<HD>;
   dim3 grid((p.n_q + 255) / 256, p.heads, p.frames);
-  attn_kernel<HD, kExpMode, V><<<grid, kThreads, Cfg<HD, V>::SMEM, stream>>>(p);
+  attn_kernel<HD, kExpMode<HD>, V><<<grid, kThreads, Cfg<HD, V>::SMEM, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? 0 : 4;
 }
 
