@@ -350,6 +350,47 @@ def sink_stream_step(torch, P, stream):
             "pool_count": st["pool_count"], "n_roll": st["n_roll"]}
 
 
+def lpm_window_step(torch, P, stream):
+    """LPM window cache with the window full: 1024 reference tokens + 3 sink + 2
+    sliding + the current chunk of 4096 tokens (25600 keys), 40 heads x 128; the
+    rotary code applied in the kernel. Timed by CUDA events around pl_lpm_step
+    alone, next to the same attention without the rotary code."""
+    R, L, heads, hd = 1024, 4096, 40, 128
+    C = heads * hd
+    g = torch.Generator(device="cuda").manual_seed(SEED)
+    lpm = P.Lpm(R, L, heads, hd)
+    rk, rv = lpm.ref_kv()
+    rk.copy_(torch.randn((R, C), device="cuda", dtype=torch.float16, generator=g))
+    rv.copy_(torch.randn((R, C), device="cuda", dtype=torch.float16, generator=g))
+    q = torch.randn((L, C), device="cuda", dtype=torch.float16, generator=g)
+    kv = torch.randn((2, L, C), device="cuda", dtype=torch.float16, generator=g)
+    out = torch.empty_like(q)
+    times = []
+    with torch.cuda.stream(stream):
+        for t in range(10):
+            kd, vd = lpm.chunk_kv()
+            kd.copy_(kv[0])
+            vd.copy_(kv[1])
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            lpm.step(q, out=out, stream=stream)
+            e1.record(stream)
+            times.append((e0, e1))
+    stream.synchronize()
+    st = lpm.state()
+    steady = [a.elapsed_time(b) for a, b in times[5:]]      # window full from step 5
+    ms = sum(steady) / len(steady)
+    # the same window without the rotary code
+    segs = [(kv[0][:R], kv[1][:R])] + [(kv[0], kv[1])] * 6
+    t_plain = _event_time(torch, lambda: P.segment_attention(q[None], segs, heads, hd,
+                                                             out=out[None], stream=stream),
+                          5, stream)
+    lpm.close()
+    fl = 4.0 * L * (R + 6 * L) * hd * heads
+    return {"ms_per_step": ms, "tflops": fl / ms / 1e9, "keys": R + 6 * L,
+            "ms_without_rotary": t_plain * 1e3, "n_sink": st["n_sink"], "n_slide": st["n_slide"]}
+
+
 def secondary_measurements(torch, P, stream, hbm_peak):
     """The other workloads' kernels, timed live (CUDA events on their stream):
     the PR-Sink block (4096 tokens x 40 heads x 128, KV own + sink + retrieved
@@ -531,6 +572,7 @@ def run_ours(args, rank, world, local_rank):
         sec = secondary_measurements(torch, P, stream, hbm_peak)
         sec["sessions_4"] = sessions_round(torch, P, wl, stream, 4, elapsed / args.steps * 1e3)
         sec["pr_sink_cache_step"] = sink_stream_step(torch, P, stream)
+        sec["lpm_window_step"] = lpm_window_step(torch, P, stream)
         line["config"]["secondary"] = sec
     clk = clocks_summary(clk_path)
     if clk is not None:

@@ -52,6 +52,14 @@ class SinkState(C.Structure):
         return {k: getattr(self, k) for k, _ in self._fields_}
 
 
+class LpmState(C.Structure):
+    _fields_ = [("chunks", C.c_int64), ("n_sink", C.c_int32), ("n_slide", C.c_int32),
+                ("last_q_pos0", C.c_int32)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
 class LayerWeights(C.Structure):
     _fields_ = [("w_qkv", vp), ("w_o", vp), ("m_q", vp), ("m_kv", vp), ("m_o", vp)]
 
@@ -105,6 +113,17 @@ _SIGS = {
     "pl_sink_block_kv": (i32, [vp, C.POINTER(vp), C.POINTER(vp)]),
     "pl_sink_step": (i32, [vp, vp, vp, vp, vp]),
     "pl_sink_get_state": (i32, [vp, C.POINTER(SinkState), vp]),
+    "pl_rope_table": (i32, [vp, i32, i32, f32, vp]),
+    "pl_rope_attention_workspace_bytes": (i32, [i32, i64, i32, i32, C.POINTER(sz)]),
+    "pl_rope_attention": (i32, [vp, i64, i32, C.POINTER(KVSegment), C.POINTER(i64), i32, i32, i32,
+                                i32, vp, i32, vp, i64, vp, sz, vp]),
+    "pl_lpm_workspace_bytes": (i32, [i32, i32, i32, i32, C.POINTER(sz)]),
+    "pl_lpm_create": (i32, [i32, i32, i32, i32, f32, vp, sz, C.POINTER(vp)]),
+    "pl_lpm_destroy": (i32, [vp]),
+    "pl_lpm_ref_kv": (i32, [vp, C.POINTER(vp), C.POINTER(vp)]),
+    "pl_lpm_chunk_kv": (i32, [vp, C.POINTER(vp), C.POINTER(vp)]),
+    "pl_lpm_step": (i32, [vp, vp, vp, vp]),
+    "pl_lpm_get_state": (i32, [vp, C.POINTER(LpmState)]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -438,4 +457,92 @@ class Sink:
     def state(self, stream=None):
         s = SinkState()
         check(lib.pl_sink_get_state(self.handle, C.byref(s), _stream(stream)), "pl_sink_get_state")
+        return s.as_dict()
+
+
+def rope_table(positions, head_dim, base=10000.0, out=None, stream=None):
+    """Device fp32 [positions, head_dim/2, 2] = (cos, sin)(pos * base^(-2i/head_dim))."""
+    import torch
+    if out is None:
+        out = torch.empty((positions, head_dim // 2, 2), dtype=torch.float32, device="cuda")
+    check(lib.pl_rope_table(_ptr(out), positions, head_dim, float(base), _stream(stream)),
+          "pl_rope_table")
+    return out
+
+
+def rope_attention(q, q_pos0, segments, seg_pos0, heads, head_dim, table, out=None, stream=None):
+    """Attention of un-rotated q [n, ld] over un-rotated (k, v) segments [len, ld], the
+    rotary code applied (once per key) at the given window positions."""
+    import torch
+    segs = (KVSegment * len(segments))()
+    pos = (i64 * len(segments))()
+    for i, ((k, v), p0) in enumerate(zip(segments, seg_pos0)):
+        segs[i] = KVSegment(_ptr(k), _ptr(v), k.shape[0], k.stride(0), 0)
+        pos[i] = int(p0)
+    if out is None:
+        out = torch.empty_like(q)
+    need = sz()
+    keys = sum(k.shape[0] for k, _ in segments)
+    check(lib.pl_rope_attention_workspace_bytes(q.shape[0], keys, heads, head_dim, C.byref(need)),
+          "pl_rope_attention_workspace_bytes")
+    ws = torch.empty(need.value, dtype=torch.uint8, device=q.device)
+    check(lib.pl_rope_attention(_ptr(q), q.stride(0), int(q_pos0), segs, pos, len(segments),
+                                q.shape[0], heads, head_dim, _ptr(table), table.shape[0],
+                                _ptr(out), out.stride(0), _ptr(ws), need.value, _stream(stream)),
+          "pl_rope_attention")
+    return out
+
+
+class Lpm:
+    """LPM window cache: reference tokens + 3 sink chunks + 2 sliding chunks (pl_lpm_*)."""
+
+    def __init__(self, ref_tokens, chunk_tokens, heads, head_dim, base=10000.0, device="cuda"):
+        import torch
+        self.ref_tokens, self.chunk_tokens = ref_tokens, chunk_tokens
+        self.heads, self.head_dim = heads, head_dim
+        need = sz()
+        check(lib.pl_lpm_workspace_bytes(ref_tokens, chunk_tokens, heads, head_dim,
+                                         C.byref(need)), "pl_lpm_workspace_bytes")
+        self.workspace = torch.empty(need.value, dtype=torch.uint8, device=device)
+        h = vp()
+        check(lib.pl_lpm_create(ref_tokens, chunk_tokens, heads, head_dim, float(base),
+                                _ptr(self.workspace), need.value, C.byref(h)), "pl_lpm_create")
+        self.handle = h
+
+    def close(self):
+        if self.handle:
+            lib.pl_lpm_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _views(self, fn, rows):
+        import torch
+        k, v = vp(), vp()
+        check(fn(self.handle, C.byref(k), C.byref(v)), fn.__name__)
+        shape = (rows, self.heads * self.head_dim)
+        return (torch.as_tensor(_DeviceArray(k.value, shape, "<f2"), device="cuda"),
+                torch.as_tensor(_DeviceArray(v.value, shape, "<f2"), device="cuda"))
+
+    def ref_kv(self):
+        return self._views(lib.pl_lpm_ref_kv, self.ref_tokens)
+
+    def chunk_kv(self):
+        return self._views(lib.pl_lpm_chunk_kv, self.chunk_tokens)
+
+    def step(self, q, out=None, stream=None):
+        import torch
+        if out is None:
+            out = torch.empty_like(q)
+        check(lib.pl_lpm_step(self.handle, _ptr(_contig(q, "q")), _ptr(out), _stream(stream)),
+              "pl_lpm_step")
+        return out
+
+    def state(self):
+        s = LpmState()
+        check(lib.pl_lpm_get_state(self.handle, C.byref(s)), "pl_lpm_get_state")
         return s.as_dict()

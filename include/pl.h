@@ -265,6 +265,71 @@ pl_status pl_sink_step(pl_sink* sink, const void* q, const float* pose, void* ou
 pl_status pl_sink_get_state(pl_sink* sink, pl_sink_state* out, void* stream);
 
 /* ------------------------------------------------------------------ *
+ * Pre-rotary KV cache with a sliding window
+ * ------------------------------------------------------------------ */
+
+/* Rotary position table (the rotary code of the LPM 1.0 write-up, section
+ * 7.4 "Pre-RoPE KV Cache"): tab[pos][i] = (cos, sin)(pos * base^(-2i / head_dim)),
+ * i < head_dim / 2, fp32 pairs computed from fp64 angles. tab: device,
+ * 8-byte aligned, positions * head_dim / 2 float pairs. */
+pl_status pl_rope_table(float* tab, int positions, int head_dim, float base, void* stream);
+
+/* Attention with the rotary code (LPM 1.0 write-up, section 7.4 "Pre-RoPE
+ * KV Cache": K/V are kept before the rotary code, which is applied by each
+ * token's position in the current window):
+ *   out = softmax(R(q) R(K_cat)^T / sqrt(head_dim)) V_cat,
+ * where R turns the pairs (2i, 2i+1) of each head by pos * theta_i; query
+ * row g sits at q_pos0 + g, row j of segment s at seg_pos0[s] + j. Q and
+ * every K are rotated once per key into the workspace (an HBM-bound pass),
+ * then the segment attention runs on the rotated copies and the caller's V.
+ * q, out: device fp16 [n_q][ld]; segments as pl_segment_attention with
+ * frame_stride 0 and ld = heads * head_dim; tab: pl_rope_table covering every
+ * position used; workspace: device, 16-byte aligned, >=
+ * pl_rope_attention_workspace_bytes(n_q, total keys, heads, head_dim). */
+pl_status pl_rope_attention_workspace_bytes(int n_q, int64_t total_keys, int heads, int head_dim,
+                                            size_t* bytes);
+pl_status pl_rope_attention(const void* q, int64_t ldq, int q_pos0, const pl_kv_segment* segs,
+                            const int64_t* seg_pos0, int n_segs, int n_q, int heads, int head_dim,
+                            const float* tab, int tab_positions, void* out, int64_t ldo,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* LPM window cache (LPM 1.0 write-up, section 7.3 "滑动窗口注意力"): a new
+ * chunk attends the reference tokens (always kept), three fixed sink chunks and the two most
+ * recent chunks, so the context stays bounded however long the session.
+ * Readings of what the write-up leaves open: the first three chunks become
+ * the sinks; later chunks slide (a full window drops its oldest); positions
+ * are the order of [reference ; sinks ; sliding oldest first ; current] in
+ * the window, so a sliding chunk's position changes as it ages and its
+ * cached (un-rotated) K is rotated again at its new position; the reference
+ * and the sinks never move and are rotated once. Chunks live in a device
+ * arena of 6 chunk blocks and never
+ * move; the caller writes each chunk's un-rotated K and V (fp16
+ * [chunk_tokens][heads*head_dim]) at the pointers pl_lpm_chunk_kv returns,
+ * and the reference tokens' once at pl_lpm_ref_kv's. */
+typedef struct pl_lpm pl_lpm;
+
+typedef struct pl_lpm_state {
+  int64_t chunks;       /* steps taken */
+  int32_t n_sink;       /* 0..3 */
+  int32_t n_slide;      /* 0..2 */
+  int32_t last_q_pos0;  /* window position of the last step's first query row, -1 before */
+} pl_lpm_state;
+
+pl_status pl_lpm_workspace_bytes(int ref_tokens, int chunk_tokens, int heads, int head_dim,
+                                 size_t* bytes);
+/* ref_tokens >= 0, chunk_tokens >= 1, head_dim in {40, 64, 80, 128, 160},
+ * rope_base > 1;
+ * workspace: device, 256-byte aligned. */
+pl_status pl_lpm_create(int ref_tokens, int chunk_tokens, int heads, int head_dim,
+                        float rope_base, void* workspace, size_t workspace_bytes, pl_lpm** out);
+pl_status pl_lpm_destroy(pl_lpm* lpm);
+pl_status pl_lpm_ref_kv(pl_lpm* lpm, void** k, void** v);
+pl_status pl_lpm_chunk_kv(pl_lpm* lpm, void** k, void** v);
+/* One chunk: q, out device fp16 [chunk_tokens][heads*head_dim] (un-rotated q). */
+pl_status pl_lpm_step(pl_lpm* lpm, const void* q, void* out, void* stream);
+pl_status pl_lpm_get_state(pl_lpm* lpm, pl_lpm_state* out);
+
+/* ------------------------------------------------------------------ *
  * Stream context: the device-resident pile and the reference bank
  * ------------------------------------------------------------------ */
 

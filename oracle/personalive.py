@@ -10,6 +10,10 @@ Sources (web pages; cited by page and section):
         conditioning paths), "TensorRT 融合" (fused graph signature).
   [LA]  LiveAnimate (iitog.ru): PR-Sink paragraph (bounded KV cache of a
         static sink block, one pose-retrieved block and three rolling slots).
+  [LPM] LPM 1.0 real-time digital actor write-up (sjmshsh.github.io):
+        sections 7.3 "滑动窗口注意力" (3 sink chunks, 2 sliding chunks,
+        reference tokens kept) and 7.4 "Pre-RoPE KV Cache" (cache K/V before
+        the rotary code, rotate by the current window position).
 
 Every function computes the plain definition in float64 with library matmuls
 as the only primitive; nothing is blocked, fused or reordered.
@@ -304,6 +308,75 @@ class PRSinkCache:
             self.rolling.append((k, v, np.asarray(pose)))
         self.blocks += 1
         return out, slot
+
+
+# ---------------------------------------------------------------------------
+# Pre-rotary KV cache with a sliding window. [LPM] sections 7.3
+# "滑动窗口注意力" (sliding-window attention) and 7.4 "Pre-RoPE KV Cache".
+# ---------------------------------------------------------------------------
+
+def rope(x: np.ndarray, pos0: int, heads: int, base: float = 10000.0) -> np.ndarray:
+    """Rotary code: in each head, the pair (2i, 2i+1) of row r turns by the
+    angle (pos0 + r) * base^(-2i / head_dim). x [n, heads*head_dim]."""
+    x = np.asarray(x, np.float64)
+    n, C = x.shape
+    hd = C // heads
+    theta = base ** (-2.0 * np.arange(hd // 2) / hd)
+    ang = (pos0 + np.arange(n, dtype=np.float64))[:, None] * theta[None, :]
+    c, s = np.cos(ang)[:, None, :], np.sin(ang)[:, None, :]
+    pairs = x.reshape(n, heads, hd // 2, 2)
+    y0 = pairs[..., 0] * c - pairs[..., 1] * s
+    y1 = pairs[..., 0] * s + pairs[..., 1] * c
+    return np.stack([y0, y1], axis=-1).reshape(n, C)
+
+
+def rope_attention(q, q_pos0, segs_k, segs_v, seg_pos0, heads, base=10000.0):
+    """Attention after the rotary code: Q at q_pos0.., segment s at seg_pos0[s].."""
+    ks = [rope(k, p, heads, base) for k, p in zip(segs_k, seg_pos0)]
+    return segment_attention(rope(q, q_pos0, heads, base), ks, segs_v, heads)
+
+
+class LPMCache:
+    """[LPM] The window of a new chunk: the reference tokens (always kept),
+    three fixed sink chunks and the two most recent chunks; K/V kept before
+    the rotary code. Readings where the write-up is silent: the first three
+    chunks become the sinks, later ones slide (a full window drops its
+    oldest); positions follow the window's order [reference ; sinks ;
+    sliding oldest first ; current], so a sliding chunk's position changes
+    as it ages and its cached K is rotated afresh every step.
+    """
+
+    SINKS, SLIDE = 3, 2
+
+    def __init__(self, ref_k, ref_v, heads, base=10000.0):
+        self.ref = (ref_k, ref_v) if ref_k is not None and len(ref_k) else None
+        self.heads, self.base = heads, base
+        self.sinks = []
+        self.slide = deque()
+        self.chunks = 0
+
+    def window(self):
+        parts = ([self.ref] if self.ref is not None else []) + self.sinks + list(self.slide)
+        pos, out = 0, []
+        for k, v in parts:
+            out.append((k, v, pos))
+            pos += len(k)
+        return out, pos
+
+    def step(self, q, k, v):
+        parts, q_pos0 = self.window()
+        ks = [p[0] for p in parts] + [k]
+        vs = [p[1] for p in parts] + [v]
+        ps = [p[2] for p in parts] + [q_pos0]
+        out = rope_attention(q, q_pos0, ks, vs, ps, self.heads, self.base)
+        if len(self.sinks) < self.SINKS:
+            self.sinks.append((k, v))
+        else:
+            if len(self.slide) == self.SLIDE:
+                self.slide.popleft()
+            self.slide.append((k, v))
+        self.chunks += 1
+        return out, q_pos0
 
 
 # ---------------------------------------------------------------------------

@@ -114,3 +114,22 @@ def test_sink_validation():
     assert L.pl_sink_create(64, 1, 64, 2, 8, None, 0, C.byref(h)) == P.PL_EINVAL
     assert L.pl_sink_create(64, 1, 64, 2, 8, C.c_void_p(256), 16, C.byref(h)) == P.PL_ENOMEM
     assert L.pl_sink_step(None, None, None, None, None) == P.PL_EINVAL
+
+
+def test_rope_and_lpm_validation():
+    import denoise_step_b200 as P
+    n = C.c_size_t()
+    L = P.lib
+    assert L.pl_lpm_workspace_bytes(1024, 4096, 40, 128, C.byref(n)) == P.PL_OK
+    # 6 chunk blocks of K and V, the reference's K and V, the rotated window, the queries, the table
+    row = 40 * 128 * 2
+    assert n.value >= (12 * 4096 + 2 * 1024 + (1024 + 6 * 4096) + 4096) * row
+    assert L.pl_lpm_workspace_bytes(1024, 4096, 40, 96, C.byref(n)) == P.PL_EUNSUPPORTED
+    assert L.pl_lpm_workspace_bytes(-1, 4096, 40, 128, C.byref(n)) == P.PL_EINVAL
+    assert L.pl_lpm_workspace_bytes(0, 0, 40, 128, C.byref(n)) == P.PL_EINVAL
+    h = C.c_void_p()
+    assert L.pl_lpm_create(16, 64, 1, 64, 10000.0, None, 0, C.byref(h)) == P.PL_EINVAL
+    assert L.pl_lpm_create(16, 64, 1, 64, 1.0, C.c_void_p(256), 1 << 40, C.byref(h)) == P.PL_EINVAL
+    assert L.pl_rope_table(None, 10, 64, 10000.0, None) == P.PL_EINVAL
+    assert L.pl_rope_table(C.c_void_p(256), 10, 63, 10000.0, None) == P.PL_EINVAL
+    assert L.pl_rope_attention_workspace_bytes(0, 10, 1, 64, C.byref(n)) == P.PL_EINVAL

@@ -449,3 +449,51 @@ def test_pr_sink_retrieval_nearest_pose_lowest_slot_on_ties():
     assert slot == 1
     _, _, slot = cache.parts(np.array([4.0, 0.0]))
     assert slot == 0
+
+
+# ------------------------------------------------------------------ rotary code and the LPM window
+
+def test_rope_hand_values_and_identity_at_zero():
+    x = np.array([[1.0, 0.0]])
+    assert np.allclose(O.rope(x, 1, heads=1), [[np.cos(1.0), np.sin(1.0)]], atol=1e-15)
+    # head_dim 4, base 100: pair 1 turns by 100^(-1/2) = 0.1 rad per position
+    y = O.rope(np.array([[0.0, 0.0, 0.0, 2.0]]), 3, heads=1, base=100.0)
+    assert np.allclose(y, [[0.0, 0.0, -2.0 * np.sin(0.3), 2.0 * np.cos(0.3)]], atol=1e-15)
+    z = S.normal(31, "rz", (1, 64))
+    assert np.array_equal(O.rope(z, 0, heads=2), z)
+
+
+def test_rope_keeps_pair_norms():
+    x = S.normal(32, "rn", (7, 2 * 64))
+    y = O.rope(x, 1000, heads=2)
+    nx = np.hypot(x[:, 0::2], x[:, 1::2])
+    ny = np.hypot(y[:, 0::2], y[:, 1::2])
+    assert np.max(np.abs(nx - ny)) < 1e-12
+
+
+def test_rope_attention_depends_only_on_relative_positions():
+    heads, C = 2, 128
+    q = S.normal(33, "q", (5, C))
+    ks = [S.normal(33, f"k{i}", (L, C)) for i, L in enumerate((6, 9))]
+    vs = [S.normal(33, f"v{i}", (L, C)) for i, L in enumerate((6, 9))]
+    a = O.rope_attention(q, 20, ks, vs, [0, 6], heads)
+    b = O.rope_attention(q, 20 + 777, ks, vs, [777, 6 + 777], heads)
+    assert np.max(np.abs(a - b)) < 1e-10
+    c = O.rope_attention(q, 21, ks, vs, [0, 6], heads)     # one position apart: differs
+    assert np.max(np.abs(a - c)) > 1e-6
+
+
+def test_lpm_window_lifecycle():
+    R, L, heads, C = 3, 4, 1, 64
+    cache = O.LPMCache(np.zeros((R, C)), np.zeros((R, C)), heads)
+    want_q_pos0 = [R, R + L, R + 2 * L, R + 3 * L, R + 4 * L, R + 5 * L, R + 5 * L, R + 5 * L]
+    for t in range(8):
+        k = np.full((L, C), float(t))
+        _, q_pos0 = cache.step(np.zeros((L, C)), k, k)
+        assert q_pos0 == want_q_pos0[t]
+    assert [int(k[0, 0]) for k, _ in cache.sinks] == [0, 1, 2]
+    assert [int(k[0, 0]) for k, _ in cache.slide] == [6, 7]
+    # chunk 7 sits right after the sinks' and chunk 6's tokens; the next step moves it
+    parts, _ = cache.window()
+    assert [(int(k[0, 0]) if len(k) == L else -1, p) for k, _, p in parts] == [
+        (-1, 0), (0, R), (1, R + L), (2, R + 2 * L), (6, R + 3 * L), (7, R + 4 * L)]
