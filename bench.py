@@ -391,6 +391,32 @@ def lpm_window_step(torch, P, stream):
             "ms_without_rotary": t_plain * 1e3, "n_sink": st["n_sink"], "n_slide": st["n_slide"]}
 
 
+def pose_front(torch, P, stream, hbm_peak):
+    """Pose path front: keypoints and dot images of a round's 4 new frames at
+    512 x 512, and of 64 frames (a 201 MB image batch, past L2) for the HBM
+    fraction. Synthetic poses (N(0, 15 deg) angles, N(0, 0.1) translations)."""
+    g = torch.Generator(device="cuda").manual_seed(SEED)
+    canon = 0.3 * torch.randn((21, 3), device="cuda", generator=g)
+    cols = [[1, 0, 0], [0, 1, 0], [0, 0, 1], [1, 1, 0], [1, 0, 1], [0, 1, 1], [0.5, 0.5, 0.5]]
+    sel = [0, 3, 5, 8, 11, 15, 20]
+    out = {}
+    for frames in (4, 64):
+        poses = torch.cat([15 * torch.randn((frames, 3), device="cuda", generator=g),
+                           0.1 * torch.randn((frames, 3), device="cuda", generator=g)], 1)
+        kps = torch.empty((frames, 7, 3), dtype=torch.float64, device="cuda")
+        img = torch.empty((frames, 3, 512, 512), dtype=torch.float32, device="cuda")
+
+        def fn():
+            P.pose_keypoints(canon, 0.9, poses, sel, out=kps, stream=stream)
+            P.pose_dots(kps, cols, 6.0, 512, 512, out=img, stream=stream)
+
+        t = _event_time(torch, fn, 10, stream)
+        byts = img.numel() * 4.0
+        out[f"frames_{frames}"] = {"us": t * 1e6, "gbs": byts / t / 1e9,
+                                   "frac_hbm": byts / t / 1e9 / hbm_peak}
+    return out
+
+
 def secondary_measurements(torch, P, stream, hbm_peak):
     """The other workloads' kernels, timed live (CUDA events on their stream):
     the PR-Sink block (4096 tokens x 40 heads x 128, KV own + sink + retrieved
@@ -573,6 +599,7 @@ def run_ours(args, rank, world, local_rank):
         sec["sessions_4"] = sessions_round(torch, P, wl, stream, 4, elapsed / args.steps * 1e3)
         sec["pr_sink_cache_step"] = sink_stream_step(torch, P, stream)
         sec["lpm_window_step"] = lpm_window_step(torch, P, stream)
+        sec["pose_front_512"] = pose_front(torch, P, stream, hbm_peak)
         line["config"]["secondary"] = sec
     clk = clocks_summary(clk_path)
     if clk is not None:

@@ -124,6 +124,9 @@ _SIGS = {
     "pl_lpm_chunk_kv": (i32, [vp, C.POINTER(vp), C.POINTER(vp)]),
     "pl_lpm_step": (i32, [vp, vp, vp, vp]),
     "pl_lpm_get_state": (i32, [vp, C.POINTER(LpmState)]),
+    "pl_pose_keypoints": (i32, [vp, f32, vp, i32, C.POINTER(i32), vp, vp]),
+    "pl_pose_ramp": (i32, [vp, vp, i32, vp, vp]),
+    "pl_pose_dots": (i32, [vp, i32, C.POINTER(f32), f32, i32, i32, vp, vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -546,3 +549,37 @@ class Lpm:
         s = LpmState()
         check(lib.pl_lpm_get_state(self.handle, C.byref(s)), "pl_lpm_get_state")
         return s.as_dict()
+
+
+def pose_keypoints(canon, scale, poses, sel, out=None, stream=None):
+    """Retargeted selected keypoints [frames, 7, 3] (fp64) of poses [frames, 6]."""
+    import torch
+    frames = poses.shape[0]
+    if out is None:
+        out = torch.empty((frames, 7, 3), dtype=torch.float64, device=poses.device)
+    s = (i32 * 7)(*[int(x) for x in sel])
+    check(lib.pl_pose_keypoints(_ptr(canon), float(scale), _ptr(_contig(poses, "poses")), frames,
+                                s, _ptr(out), _stream(stream)), "pl_pose_keypoints")
+    return out
+
+
+def pose_ramp(kps_from, kps_to, frames=12, out=None, stream=None):
+    import torch
+    if out is None:
+        out = torch.empty((frames, 7, 3), dtype=torch.float64, device=kps_from.device)
+    check(lib.pl_pose_ramp(_ptr(kps_from), _ptr(kps_to), frames, _ptr(out), _stream(stream)),
+          "pl_pose_ramp")
+    return out
+
+
+def pose_dots(kps, colours, radius, H, W, out=None, stream=None):
+    """Dot images [frames, 3, H, W] fp32 of keypoints [frames, 7, 3]."""
+    import numpy as np
+    import torch
+    frames = kps.shape[0]
+    if out is None:
+        out = torch.empty((frames, 3, H, W), dtype=torch.float32, device=kps.device)
+    col = (f32 * 21)(*[float(x) for x in np.asarray(colours, np.float32).ravel()])
+    check(lib.pl_pose_dots(_ptr(_contig(kps, "kps")), frames, col, float(radius), H, W, _ptr(out),
+                           _stream(stream)), "pl_pose_dots")
+    return out

@@ -330,6 +330,39 @@ pl_status pl_lpm_step(pl_lpm* lpm, const void* q, void* out, void* stream);
 pl_status pl_lpm_get_state(pl_lpm* lpm, pl_lpm_state* out);
 
 /* ------------------------------------------------------------------ *
+ * Pose path front
+ * ------------------------------------------------------------------ */
+
+/* PersonaLive write-up, "三条条件通路" (pose as a residual): 21 implicit 3D
+ * keypoints with pitch / yaw / roll / translation / scale; retargeting keeps
+ * the reference's canonical keypoints and scale and takes only the driving
+ * frame's rotation and half its translation; 7 of the points are drawn as
+ * coloured dots for the pose guider. Readings where the page is silent:
+ * angles in degrees, R = Rz(roll) Ry(yaw) Rx(pitch) on column vectors,
+ * keypoint = scale * R c + 0.5 t; the dot image is orthographic with x, y in
+ * [-1, 1] mapped to [0, W] x [0, H]; a pixel (centre (x + 0.5, y + 0.5))
+ * takes the colour of the last selected dot within `radius` pixels
+ * (d^2 <= r^2 in fp64), black elsewhere; the 12 prefill frames' keypoints are
+ * the 13-point ramp from the reference pose to the first driving pose, last
+ * point dropped. Keypoints are fp64. */
+#define PL_POSE_POINTS 21
+#define PL_POSE_DOTS 7
+
+/* kps[f][j] = scale * R(pose_f) canon[sel[j]] + 0.5 t_f. canon: device fp32
+ * [21][3]; poses: device fp32 [frames][6] = (pitch, yaw, roll, tx, ty, tz);
+ * sel: host int32 [7] (indices < 21); kps: device double [frames][7][3]. */
+pl_status pl_pose_keypoints(const float* canon, float scale, const float* poses, int frames,
+                            const int32_t* sel, double* kps, void* stream);
+/* out[k] = from + (k / frames)(to - from), k < frames: the prefill ramp
+ * (frames = 12). from, to: device double [7][3]; out: device [frames][7][3]. */
+pl_status pl_pose_ramp(const double* kps_from, const double* kps_to, int frames, double* out,
+                       void* stream);
+/* Dot images: image device fp32 [frames][3][H][W] from kps [frames][7][3];
+ * colours: host fp32 [7][3]. */
+pl_status pl_pose_dots(const double* kps, int frames, const float* colours, float radius, int H,
+                       int W, float* image, void* stream);
+
+/* ------------------------------------------------------------------ *
  * Stream context: the device-resident pile and the reference bank
  * ------------------------------------------------------------------ */
 

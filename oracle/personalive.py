@@ -397,6 +397,62 @@ def prefill_motion(ref_motion, drive0_motion, frames: int = 12) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Pose path front. [PL] "三条条件通路" (pose as a residual): 21 implicit 3D
+# keypoints with pitch / yaw / roll / translation / scale; retargeting keeps
+# the reference's canonical keypoints and scale, takes only the driving
+# rotation and half its translation; 7 of the 21 points are drawn as coloured
+# dots. Readings where the page is silent (listed in the design doc): angles in
+# degrees, R = Rz(roll) Ry(yaw) Rx(pitch) acting on column vectors; keypoint
+# = scale * R c + 0.5 t; the dot image is orthographic with x, y in [-1, 1]
+# mapped to [0, W] x [0, H] (z dropped); a pixel (centre (x + 0.5, y + 0.5))
+# takes the colour of the last of the 7 dots whose centre lies within the
+# radius (d^2 <= r^2, fp64), black elsewhere; the prefill frames' keypoints
+# are the 13-point ramp from the reference pose to the first driving pose,
+# last point dropped (as the motion ramp).
+# ---------------------------------------------------------------------------
+
+def rotation(pitch: float, yaw: float, roll: float) -> np.ndarray:
+    """R = Rz(roll) @ Ry(yaw) @ Rx(pitch), angles in degrees."""
+    p, y, r = np.radians([pitch, yaw, roll])
+    rx = np.array([[1, 0, 0], [0, np.cos(p), -np.sin(p)], [0, np.sin(p), np.cos(p)]])
+    ry = np.array([[np.cos(y), 0, np.sin(y)], [0, 1, 0], [-np.sin(y), 0, np.cos(y)]])
+    rz = np.array([[np.cos(r), -np.sin(r), 0], [np.sin(r), np.cos(r), 0], [0, 0, 1]])
+    return rz @ ry @ rx
+
+
+def retarget(canon: np.ndarray, scale: float, pose) -> np.ndarray:
+    """Keypoints [21, 3] = scale * R(pose) c + 0.5 t: the reference's canonical
+    points and scale, the driving frame's rotation, half its translation.
+    pose = (pitch, yaw, roll, tx, ty, tz)."""
+    pose = np.asarray(pose, np.float64)
+    R = rotation(*pose[:3])
+    return scale * (np.asarray(canon, np.float64) @ R.T) + 0.5 * pose[3:6][None, :]
+
+
+def dot_centres(kps: np.ndarray, sel, H: int, W: int) -> np.ndarray:
+    """Pixel coordinates [7, 2] (x, y) of the selected keypoints."""
+    k = np.asarray(kps, np.float64)[list(sel)]
+    return np.stack([(k[:, 0] + 1.0) * 0.5 * W, (k[:, 1] + 1.0) * 0.5 * H], axis=1)
+
+
+def dot_image(centres: np.ndarray, colours: np.ndarray, radius: float, H: int, W: int):
+    """[3, H, W] fp32: each pixel the colour of the last dot covering it."""
+    img = np.zeros((3, H, W), np.float32)
+    yy, xx = np.meshgrid(np.arange(H) + 0.5, np.arange(W) + 0.5, indexing="ij")
+    for (cx, cy), col in zip(np.asarray(centres, np.float64), np.asarray(colours, np.float32)):
+        inside = (xx - cx) ** 2 + (yy - cy) ** 2 <= float(radius) ** 2
+        img[:, inside] = col[:, None]
+    return img
+
+
+def prefill_keypoints(kps_ref: np.ndarray, kps_drive0: np.ndarray, frames: int = 12):
+    """Keypoints of the prefill frames: the 13-point ramp, last point dropped."""
+    a = np.asarray(kps_ref, np.float64).ravel()
+    b = np.asarray(kps_drive0, np.float64).ravel()
+    return interpolate(a, b, frames + 1)[:-1].reshape(frames, *np.shape(kps_ref))
+
+
+# ---------------------------------------------------------------------------
 # The round's state machine (explicit deque). [PL] "流式金字塔去噪".
 # ---------------------------------------------------------------------------
 

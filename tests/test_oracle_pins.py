@@ -497,3 +497,43 @@ def test_lpm_window_lifecycle():
     parts, _ = cache.window()
     assert [(int(k[0, 0]) if len(k) == L else -1, p) for k, _, p in parts] == [
         (-1, 0), (0, R), (1, R + L), (2, R + 2 * L), (6, R + 3 * L), (7, R + 4 * L)]
+
+
+# ------------------------------------------------------------------ pose path front ([PL] 三条条件通路)
+
+def test_rotation_axes_and_orthogonality():
+    assert np.array_equal(O.rotation(0, 0, 0), np.eye(3))
+    ex, ey = np.array([1.0, 0, 0]), np.array([0, 1.0, 0])
+    assert np.allclose(O.rotation(0, 0, 90) @ ex, [0, 1, 0], atol=1e-15)    # roll: x -> y
+    assert np.allclose(O.rotation(90, 0, 0) @ ey, [0, 0, 1], atol=1e-15)    # pitch: y -> z
+    assert np.allclose(O.rotation(0, 90, 0) @ ex, [0, 0, -1], atol=1e-15)   # yaw: x -> -z
+    R = O.rotation(17.0, -33.0, 71.0)
+    assert np.allclose(R @ R.T, np.eye(3), atol=1e-15) and abs(np.linalg.det(R) - 1) < 1e-14
+
+
+def test_retarget_keeps_canonical_points_and_scale_halves_translation():
+    c = S.normal(41, "canon", (21, 3))
+    got = O.retarget(c, 1.7, (0, 0, 0, 0.2, -0.4, 3.0))
+    assert np.allclose(got, 1.7 * c + [0.1, -0.2, 1.5], atol=1e-15)
+    # rotation only enters through R: distances between points scale by 1.7
+    r = O.retarget(c, 1.7, (10, 20, 30, 0, 0, 0))
+    assert np.allclose(np.linalg.norm(r[3] - r[5]), 1.7 * np.linalg.norm(c[3] - c[5]), atol=1e-14)
+
+
+def test_dot_image_disc_and_painter_order():
+    col = np.array([[1, 0, 0], [0, 1, 0]], np.float32)
+    # a dot on a pixel centre: radius 0.5 covers that pixel, radius 1 its 4 neighbours too
+    img = O.dot_image(np.array([[3.5, 2.5]]), col[:1], 0.5, 6, 8)
+    assert img[0].sum() == 1 and img[0, 2, 3] == 1
+    img = O.dot_image(np.array([[3.5, 2.5]]), col[:1], 1.0, 6, 8)
+    assert img[0].sum() == 5 and img[0, 1, 3] == 1 and img[0, 2, 4] == 1 and img[0, 1, 4] == 0
+    # overlapping dots: the later one wins where both cover
+    img = O.dot_image(np.array([[3.5, 2.5], [4.5, 2.5]]), col, 1.0, 6, 8)
+    assert img[1, 2, 4] == 1 and img[0, 2, 4] == 0 and img[0, 2, 2] == 1
+
+
+def test_prefill_keypoints_ramp():
+    a, b = S.normal(42, "a", (7, 3)), S.normal(42, "b", (7, 3))
+    k = O.prefill_keypoints(a, b)
+    assert k.shape == (12, 7, 3) and np.array_equal(k[0], a)
+    assert np.allclose(k[11] + (k[11] - k[10]), b, atol=1e-14)     # the dropped 13th point
