@@ -71,21 +71,30 @@ __global__ void pose_dots_kernel(const double* __restrict__ kps, int frames, Dot
                                  double r2, int H, int W, float* __restrict__ image) {
   const int f = blockIdx.z;
   __shared__ double cx[kDots], cy[kDots];
+  __shared__ float fx[kDots], fy[kDots];
   if (threadIdx.x < kDots) {
     const double* k = kps + (static_cast<int64_t>(f) * kDots + threadIdx.x) * 3;
     cx[threadIdx.x] = __dmul_rn(__dmul_rn(__dadd_rn(k[0], 1.0), 0.5), static_cast<double>(W));
     cy[threadIdx.x] = __dmul_rn(__dmul_rn(__dadd_rn(k[1], 1.0), 0.5), static_cast<double>(H));
+    fx[threadIdx.x] = static_cast<float>(cx[threadIdx.x]);
+    fy[threadIdx.x] = static_cast<float>(cy[threadIdx.x]);
   }
   __syncthreads();
+  // a pixel farther than radius + 1 from a centre in either axis (fp32, far
+  // beyond its rounding) cannot pass the exact test: skip the fp64 work there
+  const float reach = static_cast<float>(sqrt(r2)) + 1.f;
   const int64_t plane = static_cast<int64_t>(H) * W;
   float* img = image + static_cast<int64_t>(f) * 3 * plane;
-  for (int64_t p = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; p < plane;
-       p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int y = static_cast<int>(p / W), x = static_cast<int>(p - static_cast<int64_t>(y) * W);
+  // plane < 2^31 (checked on the host): 32-bit pixel indices and division
+  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < plane; p += gridDim.x * blockDim.x) {
+    const int y = p / W, x = p - y * W;
     const double px = x + 0.5, py = y + 0.5;
     int hit = -1;
 #pragma unroll
     for (int j = 0; j < kDots; ++j) {
+      if (fabsf(static_cast<float>(px) - fx[j]) > reach ||
+          fabsf(static_cast<float>(py) - fy[j]) > reach)
+        continue;
       const double dx = __dsub_rn(px, cx[j]), dy = __dsub_rn(py, cy[j]);
       if (__dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy)) <= r2) hit = j;
     }
@@ -125,14 +134,17 @@ pl_status pl_pose_ramp(const double* kps_from, const double* kps_to, int frames,
 pl_status pl_pose_dots(const double* kps, int frames, const float* colours, float radius, int H,
                        int W, float* image, void* stream) {
   if (!kps || !colours || !image || frames < 1 || frames > 65535) return PL_EINVAL;
-  if (H < 1 || W < 1 || static_cast<int64_t>(H) * W > (1ll << 31)) return PL_EINVAL;
+  if (H < 1 || W < 1 || static_cast<int64_t>(H) * W >= (1ll << 31) - 65536) return PL_EINVAL;
   if (!(radius >= 0.f) || !std::isfinite(radius)) return PL_EINVAL;
   DotParams dp{};
   for (int j = 0; j < kDots; ++j)
     for (int c = 0; c < 3; ++c) dp.colour[j][c] = colours[3 * j + c];
+  // about 8 blocks per SM in all, so each thread covers many pixels and the
+  // per-block set-up (the 7 centres) is paid rarely
   const int64_t plane = static_cast<int64_t>(H) * W;
   int64_t bx = (plane + 255) / 256;
-  if (bx > 148 * 8) bx = 148 * 8;
+  const int64_t cap = (148 * 8 + frames - 1) / frames;
+  if (bx > cap) bx = cap;
   const double r = radius;
   const dim3 grid(static_cast<unsigned>(bx), 1, frames);
   pose_dots_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(kps, frames, dp, r * r, H,
