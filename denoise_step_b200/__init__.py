@@ -101,6 +101,8 @@ _SIGS = {
     "pl_pyramid_ddim_step": (i32, [vp, vp, vp, vp]),
     "pl_ctx_bank_check": (i32, [vp, vp, i32, vp, vp, vp, vp]),
     "pl_stream_round": (i32, [vp, vp, vp, C.POINTER(vp), vp, vp, vp, C.POINTER(vp), vp]),
+    "pl_host_staging_bytes": (i32, [C.POINTER(Config), C.POINTER(sz)]),
+    "pl_stream_round_host": (i32, [vp, vp, sz, vp, vp, C.POINTER(vp), vp, vp, vp]),
     "pl_get_state": (i32, [vp, C.POINTER(State), vp]),
     "pl_get_session_state": (i32, [vp, i32, C.POINTER(State), vp]),
     "pl_get_motion_bank": (i32, [vp, vp, C.POINTER(C.c_int32), vp]),
@@ -384,6 +386,26 @@ class Stream:
         check(lib.pl_stream_round(self.handle, _ptr(new_noise), _ptr(new_motion), hp, _ptr(eps),
                                   _ptr(out_frames), _ptr(appended), lo, _stream(stream)),
               "pl_stream_round")
+
+    def round_host(self, h_noise, h_motion, h_hidden, h_eps, h_out_frames, stream=None):
+        """One round from pinned host tensors to a pinned host tensor (asynchronous:
+        h_out_frames is valid once `stream` is synchronised). The device staging the
+        C call needs is allocated on first use and kept with the stream."""
+        import torch
+        if getattr(self, "_staging", None) is None:
+            need = sz()
+            check(lib.pl_host_staging_bytes(C.byref(self.cfg), C.byref(need)),
+                  "pl_host_staging_bytes")
+            self._staging = torch.empty(need.value, dtype=torch.uint8,
+                                        device=self.workspace.device)
+        for t in [h_noise, h_motion, h_eps, h_out_frames, *h_hidden]:
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError("round_host takes contiguous host tensors")
+        hp = _ptr_array(h_hidden) if self.cfg.n_layers else None
+        check(lib.pl_stream_round_host(self.handle, _ptr(self._staging), self._staging.numel(),
+                                       _ptr(h_noise), _ptr(h_motion), hp, _ptr(h_eps),
+                                       _ptr(h_out_frames), _stream(stream)),
+              "pl_stream_round_host")
 
     def state(self, stream=None, session=0):
         s = State()

@@ -75,11 +75,22 @@ struct pl_ctx {
   pl_layer_weights w[PL_MAX_LAYERS];
   const void* ref_feats[PL_MAX_LAYERS];
   const void* anchor_feats[3][PL_MAX_LAYERS];
-  // captured round
-  cudaGraph_t graph;
-  cudaGraphExec_t exec;
-  const void* key[64];
-  int key_n;
+  // captured rounds, one per pointer set (two: the host path alternates
+  // between its staging sets)
+  struct GraphSlot {
+    cudaGraph_t graph;
+    cudaGraphExec_t exec;
+    const void* key[64];
+    int key_n;
+    uint64_t last_use;
+  } graphs[2];
+  uint64_t graph_tick;
+  // host path: copy stream, staging-set events, rounds issued
+  cudaStream_t copy_stream;
+  cudaEvent_t ev_in[2];     // set b's inputs are on the device
+  cudaEvent_t ev_free[2];   // the round reading set b is done
+  bool free_pending[2];
+  int64_t host_rounds;
 };
 
 namespace {
@@ -280,12 +291,51 @@ pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
   return PL_OK;
 }
 
+void drop_slot(pl_ctx::GraphSlot& g) {
+  if (g.exec) cudaGraphExecDestroy(g.exec);
+  if (g.graph) cudaGraphDestroy(g.graph);
+  g.exec = nullptr;
+  g.graph = nullptr;
+  g.key_n = 0;
+}
+
 void drop_graph(pl_ctx* ctx) {
-  if (ctx->exec) cudaGraphExecDestroy(ctx->exec);
-  if (ctx->graph) cudaGraphDestroy(ctx->graph);
-  ctx->exec = nullptr;
-  ctx->graph = nullptr;
-  ctx->key_n = 0;
+  for (auto& g : ctx->graphs) drop_slot(g);
+}
+
+// Staging of the host path: two sets, each the inputs of one round and its
+// x0 frames. With base == nullptr only the size of both sets is computed.
+struct HostSet {
+  float* noise;                      // [S][4][4][H][W]
+  float* motion;                     // [S][4][512]
+  void* hidden[PL_MAX_LAYERS];       // fp16 [S][16][N_l][C_l]
+  float* eps;                        // [S][16][4][H][W]
+  float* out;                        // [S][4][4][H][W]
+  size_t hidden_bytes[PL_MAX_LAYERS];
+};
+
+size_t host_layout(const pl_config& c, uint8_t* base, int set, HostSet* hs) {
+  const int64_t S = c.sessions > 0 ? c.sessions : 1;
+  const int64_t fe = static_cast<int64_t>(c.latent_c) * c.latent_h * c.latent_w;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> uint8_t* {
+    uint8_t* q = base ? base + off : nullptr;
+    off += align_up(bytes);
+    return q;
+  };
+  HostSet h{};
+  for (int b = 0; b <= set; ++b) {
+    h.noise = reinterpret_cast<float*>(take(sizeof(float) * S * 4 * fe));
+    h.motion = reinterpret_cast<float*>(take(sizeof(float) * S * 4 * 512));
+    for (int l = 0; l < c.n_layers; ++l) {
+      h.hidden_bytes[l] = sizeof(__half) * S * 16 * c.layer_tokens[l] * c.layer_channels[l];
+      h.hidden[l] = take(h.hidden_bytes[l]);
+    }
+    h.eps = reinterpret_cast<float*>(take(sizeof(float) * S * 16 * fe));
+    h.out = reinterpret_cast<float*>(take(sizeof(float) * S * 4 * fe));
+  }
+  if (hs) *hs = h;
+  return off;
 }
 
 }  // namespace
@@ -557,6 +607,15 @@ pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_
 pl_status pl_ctx_destroy(pl_ctx* ctx) {
   if (!ctx) return PL_OK;
   drop_graph(ctx);
+  for (int b = 0; b < 2; ++b) {
+    if (ctx->ev_in[b]) cudaEventDestroy(ctx->ev_in[b]);
+    if (ctx->ev_free[b]) cudaEventDestroy(ctx->ev_free[b]);
+  }
+  if (ctx->copy_stream) {
+    // the staging the copies write belongs to the caller: finish them first
+    cudaStreamSynchronize(ctx->copy_stream);
+    cudaStreamDestroy(ctx->copy_stream);
+  }
   delete ctx;
   return PL_OK;
 }
@@ -667,10 +726,18 @@ pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_
     key[kn++] = hidden[l];
     key[kn++] = layer_out ? layer_out[l] : nullptr;
   }
-  bool hit = ctx->exec && ctx->key_n == kn;
-  for (int i = 0; hit && i < kn; ++i) hit = ctx->key[i] == key[i];
-  if (!hit) {
-    drop_graph(ctx);
+  pl_ctx::GraphSlot* slot = nullptr;
+  for (auto& g : ctx->graphs) {
+    bool hit = g.exec && g.key_n == kn;
+    for (int i = 0; hit && i < kn; ++i) hit = g.key[i] == key[i];
+    if (hit) slot = &g;
+  }
+  if (!slot) {
+    // replace the empty or least recently used capture
+    slot = &ctx->graphs[0];
+    for (auto& g : ctx->graphs)
+      if (!g.exec || (slot->exec && g.last_use < slot->last_use)) slot = &g;
+    drop_slot(*slot);
     if (cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
       return PL_ECUDA;
     const pl_status r = enqueue_round(ctx, a, s);
@@ -681,16 +748,78 @@ pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_
       return r;
     }
     if (e != cudaSuccess || !g) return PL_ECUDA;
-    if (cudaGraphInstantiate(&ctx->exec, g, 0) != cudaSuccess) {
+    if (cudaGraphInstantiate(&slot->exec, g, 0) != cudaSuccess) {
       cudaGraphDestroy(g);
-      ctx->exec = nullptr;
+      slot->exec = nullptr;
       return PL_ECUDA;
     }
-    ctx->graph = g;
-    std::memcpy(ctx->key, key, sizeof(const void*) * kn);
-    ctx->key_n = kn;
+    slot->graph = g;
+    std::memcpy(slot->key, key, sizeof(const void*) * kn);
+    slot->key_n = kn;
   }
-  return from_cuda(cudaGraphLaunch(ctx->exec, s));
+  slot->last_use = ++ctx->graph_tick;
+  return from_cuda(cudaGraphLaunch(slot->exec, s));
+}
+
+pl_status pl_host_staging_bytes(const pl_config* cfg, size_t* bytes) {
+  if (!bytes) return PL_EINVAL;
+  const pl_status v = validate_config(cfg);
+  if (v) return v;
+  *bytes = host_layout(*cfg, nullptr, 1, nullptr);
+  return PL_OK;
+}
+
+pl_status pl_stream_round_host(pl_ctx* ctx, void* staging, size_t staging_bytes,
+                               const float* h_noise, const float* h_motion,
+                               const void* const* h_hidden, const float* h_eps,
+                               float* h_out_frames, void* stream) {
+  if (!ctx || !staging || !h_noise || !h_motion || !h_eps || !h_out_frames) return PL_EINVAL;
+  if (!ctx->initialised) return PL_ESTATE;
+  const pl_config& c = ctx->cfg;
+  const int L = c.n_layers;
+  if (L > 0 && !h_hidden) return PL_EINVAL;
+  for (int l = 0; l < L; ++l)
+    if (!h_hidden[l]) return PL_EINVAL;
+  if (reinterpret_cast<uintptr_t>(staging) % kAlign) return PL_EINVAL;
+  if (staging_bytes < host_layout(c, nullptr, 1, nullptr)) return PL_ENOMEM;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!ctx->copy_stream) {
+    if (cudaStreamCreateWithFlags(&ctx->copy_stream, cudaStreamNonBlocking) != cudaSuccess)
+      return PL_ECUDA;
+    for (int b = 0; b < 2; ++b) {
+      if (cudaEventCreateWithFlags(&ctx->ev_in[b], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&ctx->ev_free[b], cudaEventDisableTiming) != cudaSuccess)
+        return PL_ECUDA;
+    }
+  }
+  const int b = static_cast<int>(ctx->host_rounds & 1);
+  HostSet h;
+  host_layout(c, static_cast<uint8_t*>(staging), b, &h);
+  const int64_t S = ctx->sessions;
+  const size_t fe = static_cast<size_t>(ctx->frame_elems);
+  cudaStream_t cs = ctx->copy_stream;
+  // set b is refilled once the round that last read it (two calls ago) is done
+  if (ctx->free_pending[b] && cudaStreamWaitEvent(cs, ctx->ev_free[b], 0) != cudaSuccess)
+    return PL_ECUDA;
+  cudaError_t e = cudaMemcpyAsync(h.noise, h_noise, sizeof(float) * S * 4 * fe,
+                                  cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(h.motion, h_motion, sizeof(float) * S * 4 * 512, cudaMemcpyHostToDevice, cs);
+  for (int l = 0; l < L && e == cudaSuccess; ++l)
+    e = cudaMemcpyAsync(h.hidden[l], h_hidden[l], h.hidden_bytes[l], cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(h.eps, h_eps, sizeof(float) * S * 16 * fe, cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess) e = cudaEventRecord(ctx->ev_in[b], cs);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ctx->ev_in[b], 0);
+  if (e != cudaSuccess) return PL_ECUDA;
+  const pl_status r = pl_stream_round(ctx, h.noise, h.motion, h.hidden, h.eps, h.out, nullptr,
+                                      nullptr, stream);
+  if (r != PL_OK) return r;
+  if (cudaEventRecord(ctx->ev_free[b], s) != cudaSuccess) return PL_ECUDA;
+  ctx->free_pending[b] = true;
+  ++ctx->host_rounds;
+  return from_cuda(cudaMemcpyAsync(h_out_frames, h.out, sizeof(float) * S * 4 * fe,
+                                   cudaMemcpyDeviceToHost, s));
 }
 
 pl_status pl_get_session_state(pl_ctx* ctx, int session, pl_state* out, void* stream) {

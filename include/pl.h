@@ -481,6 +481,37 @@ pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_
                           const void* const* hidden, const float* eps, float* out_frames,
                           uint8_t* appended, void* const* layer_out, void* stream);
 
+/* Host-buffer round: the serving boundary of the PersonaLive write-up,
+ * "在线链路" (frames arrive from the host, four at a time, one forward per
+ * four, decoded frames go back to the host), overlapped in the manner of the
+ * LPM 1.0 page, section 7.5 (the steady rate is that of the slowest stage, so
+ * the transfer of round k + 1 runs under the compute of round k).
+ *
+ * pl_host_staging_bytes: device staging the host path needs: two sets, each
+ * holding one round's inputs and its x0 frames (about 2 x 0.4 GB per session
+ * at the 512 x 512 geometry).
+ *
+ * pl_stream_round_host: the same round as pl_stream_round with
+ * h_noise [S][4][4][H][W] fp32, h_motion [S][4][512] fp32, h_hidden (host
+ * array [n_layers] of host fp16 [S][16][N_l][C_l]) and h_eps
+ * [S][16][4][H][W] fp32 in host memory, and the x0 frames returned to
+ * h_out_frames [S][4][4][H][W] fp32 in host memory. The inputs are copied on
+ * a copy stream the context owns into staging set (call count mod 2) of
+ * `staging` (device, 256-byte aligned, >= pl_host_staging_bytes, owned by the
+ * caller and used by nothing else while the context lives), the round then
+ * runs on `stream` and the frames are copied back on `stream`. Asynchronous
+ * like cudaMemcpyAsync: the host buffers must be pinned for the copies to
+ * overlap (pageable memory works but serialises), must stay unchanged until
+ * the call's work is done, and h_out_frames is valid once `stream` has been
+ * synchronised. Returns PL_EINVAL for a NULL or misaligned argument,
+ * PL_ENOMEM for too small a staging buffer, PL_ESTATE before pl_bank_init,
+ * PL_ECUDA when a copy or launch fails to enqueue. */
+pl_status pl_host_staging_bytes(const pl_config* cfg, size_t* bytes);
+pl_status pl_stream_round_host(pl_ctx* ctx, void* staging, size_t staging_bytes,
+                               const float* h_noise, const float* h_motion,
+                               const void* const* h_hidden, const float* h_eps,
+                               float* h_out_frames, void* stream);
+
 /* Synchronise `stream` and copy the state of session 0 to *out. */
 pl_status pl_get_state(pl_ctx* ctx, pl_state* out, void* stream);
 

@@ -92,6 +92,29 @@ def test_sessions_scale_the_workspace():
         assert P.lib.pl_workspace_bytes(C.byref(cfg), C.byref(n)) == P.PL_EINVAL
 
 
+def test_host_staging_size_and_validation():
+    import denoise_step_b200 as P
+    import synthetic as S
+    layers = [(side * side, c) for _, side, c in S.LAYERS]
+    n = C.c_size_t()
+    cfg = P.make_config((64, 64), layers)
+    assert P.lib.pl_host_staging_bytes(C.byref(cfg), C.byref(n)) == P.PL_OK
+    # two sets of: noise 4 frames, motion 4 x 512, hidden 16 frames per layer
+    # (fp16), eps 16 frames, x0 4 frames; each region 256-byte aligned
+    fe = 4 * 64 * 64
+    per_set = 4 * (4 * fe + 4 * 512 + 16 * fe + 4 * fe) + sum(2 * 16 * N * c for N, c in layers)
+    assert 2 * per_set <= n.value < 2 * per_set + 2 * (4 + len(layers)) * 256
+    n2 = C.c_size_t()
+    cfg2 = P.make_config((64, 64), layers, sessions=2)
+    assert P.lib.pl_host_staging_bytes(C.byref(cfg2), C.byref(n2)) == P.PL_OK
+    assert abs(n2.value - 2 * n.value) < 2 * (4 + len(layers)) * 256
+    bad = P.make_config((64, 64), [(4096, 320)], heads=7)
+    assert P.lib.pl_host_staging_bytes(C.byref(bad), C.byref(n)) == P.PL_EINVAL
+    assert P.lib.pl_host_staging_bytes(C.byref(cfg), None) == P.PL_EINVAL
+    assert P.lib.pl_stream_round_host(None, None, 0, None, None, None, None, None,
+                                      None) == P.PL_EINVAL
+
+
 def test_round_before_init_is_a_state_error():
     import denoise_step_b200 as P
     # a null context is rejected before any device work

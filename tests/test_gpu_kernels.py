@@ -68,6 +68,32 @@ def test_segment_attention_peaky_scores(P):
     assert mx <= 3e-2 and rel < 1e-2, (mx, mean, rel)
 
 
+@pytest.mark.parametrize("hd", [40, 80, 128, 160])
+@pytest.mark.parametrize("shape", ["ramp", "spikes"])
+def test_segment_attention_growing_max(P, hd, shape):
+    # the row maximum keeps growing along the keys, so later KV tiles overflow
+    # the running maximum by far more than 2^8: "ramp" raises the key scale
+    # from 0.25 to 8 (scores up to ~40 in log2 units), "spikes" puts keys 64x
+    # larger into a few late tiles (scores past 128 in log2 units, beyond the
+    # range of a plain exponent-field exp2)
+    F, Nq, heads = 1, 160, 2
+    Cc = heads * hd
+    L = 700
+    q = S.normal(43, f"q{hd}", (F, Nq, Cc), 1.0, np.float16)
+    k = S.normal(43, f"k{hd}", (F, L, Cc), 1.0, np.float64)
+    if shape == "ramp":
+        k *= np.geomspace(0.25, 8.0, L)[None, :, None]
+    else:
+        k[:, 300::97, :] *= 64.0
+    k = k.astype(np.float16)
+    v = S.normal(43, f"v{hd}", (F, L, Cc), 1.0, np.float16)
+    got = host(P.segment_attention(dev(q), [(dev(k), dev(v))], heads, hd)).astype(np.float64)
+    want = O.segment_attention(q[0], [k[0]], [v[0]], heads)
+    assert np.all(np.isfinite(got[0]))
+    mx, mean, rel = attn_errors(got[0], want)
+    assert mx <= 3e-2 and rel < 1e-2, (mx, mean, rel)
+
+
 # ------------------------------------------------------------------ reference attention layer
 
 def _ref_case(seed, F, N, C, n_bank, scale=1.0):

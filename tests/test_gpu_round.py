@@ -122,6 +122,45 @@ def test_tiny_rounds_match_oracle(P, walk_sigma):
     st.close()
 
 
+def test_host_round_matches_device_round(P):
+    # the host-buffer round (inputs copied on the context's copy stream into
+    # two alternating staging sets, x0 frames copied back) gives the device
+    # round's frames bit for bit, with four rounds enqueued back to back
+    # before a single synchronisation
+    case = Case(S.SEEDS["tiny"], [("m", 8, 1280)], 8, 8, 3.0)
+    st_a, _, _ = _setup(P, case)
+    st_b, _, _ = _setup(P, Case(S.SEEDS["tiny"], [("m", 8, 1280)], 8, 8, 3.0))
+    stream = torch.cuda.Stream()
+    ins = []
+    for r in range(1, 5):
+        hidden, noise, eps = case.round_inputs(r)
+        ins.append((hidden, noise, case.next_motion(r), eps))
+    want = []
+    out = torch.empty((4, 4, 8, 8), dtype=torch.float32, device="cuda")
+    for hidden, noise, mot, eps in ins:
+        d_args = (dev(noise), dev(mot), [dev(h) for h in hidden], dev(eps))
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            st_a.round(*d_args, out, stream=stream)
+        stream.synchronize()
+        want.append(host(out).copy())
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    h_in = [([pin(h) for h in hidden], pin(noise), pin(mot), pin(eps))
+            for hidden, noise, mot, eps in ins]
+    h_out = [torch.full((4, 4, 8, 8), float("nan"), dtype=torch.float32).pin_memory() for _ in ins]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for (hh, hn, hm, he), ho in zip(h_in, h_out):
+            st_b.round_host(hn, hm, hh, he, ho, stream=stream)
+    stream.synchronize()
+    for r, (w, ho) in enumerate(zip(want, h_out)):
+        assert np.array_equal(ho.numpy(), w), r
+    assert st_a.state() == st_b.state()
+    assert st_b.device_status() == 0
+    st_a.close()
+    st_b.close()
+
+
 def test_full_geometry_rounds_spot_checked(P):
     # 16 reference-attention layers in the SD-UNet layout, bank x4 after round 1,
     # DDIM on 16x4x64x64, bank check; sampled rows of one layer per level
