@@ -355,11 +355,20 @@ __global__ void __launch_bounds__(128) motion_attn_kernel(const float* __restric
   for (int r = 0; r < R; ++r)
 #pragma unroll
     for (int j = 0; j < 32; ++j) s[r][j] = 0.f;
+  // the dimension loop stays rolled (a fully unrolled one overflows the
+  // instruction cache); the next four dimensions of q are in flight while
+  // these are used
+  float4 an[R];
 #pragma unroll
+  for (int r = 0; r < R; ++r) an[r] = *reinterpret_cast<const float4*>(qr[r]);
+#pragma unroll 1
   for (int d0 = 0; d0 < HD; d0 += 4) {
     float4 a[R];
 #pragma unroll
-    for (int r = 0; r < R; ++r) a[r] = *reinterpret_cast<const float4*>(qr[r] + d0);
+    for (int r = 0; r < R; ++r) {
+      a[r] = an[r];
+      if (d0 + 4 < HD) an[r] = *reinterpret_cast<const float4*>(qr[r] + d0 + 4);
+    }
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const float4 k = *reinterpret_cast<const float4*>(&sk[j][d0]);
@@ -386,7 +395,7 @@ __global__ void __launch_bounds__(128) motion_attn_kernel(const float* __restric
     inv[r] = 1.f / l;
   }
   __half* orow = out + (static_cast<int64_t>(f) * N + n0) * ldo + h * HD;
-#pragma unroll
+#pragma unroll 1
   for (int d0 = 0; d0 < HD; d0 += 8) {
     float o[R][8];
 #pragma unroll
@@ -417,7 +426,8 @@ __global__ void __launch_bounds__(128) motion_attn_kernel(const float* __restric
 }
 
 // One thread per (query row, head): 32 scores in registers, smem-resident
-// K/V of the frame and head (fp32), softmax in fp32 (head_dim >= 80).
+// K/V of the frame and head (fp32), softmax in fp32 (head_dim >= 80). The
+// dimension loops stay rolled, as in the kernel above.
 template <int HD>
 __global__ void __launch_bounds__(128) motion_attn_row_kernel(const float* __restrict__ q, int64_t ldq,
                                                           const float* __restrict__ kv, int N,
@@ -439,8 +449,11 @@ __global__ void __launch_bounds__(128) motion_attn_row_kernel(const float* __res
   float s[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) s[j] = 0.f;
+  float4 qn = *reinterpret_cast<const float4*>(qr);
+#pragma unroll 1
   for (int d0 = 0; d0 < HD; d0 += 4) {
-    const float4 qv = *reinterpret_cast<const float4*>(qr + d0);
+    const float4 qv = qn;
+    if (d0 + 4 < HD) qn = *reinterpret_cast<const float4*>(qr + d0 + 4);
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       s[j] = fmaf(qv.x, sk[j][d0], s[j]);
@@ -463,6 +476,7 @@ __global__ void __launch_bounds__(128) motion_attn_row_kernel(const float* __res
   }
   const float inv = 1.f / sum;
   __half* orow = out + (static_cast<int64_t>(f) * N + n) * ldo + h * HD;
+#pragma unroll 1
   for (int d0 = 0; d0 < HD; d0 += 8) {
     float o[8];
 #pragma unroll
