@@ -11,12 +11,18 @@
 //                                 MN-major) from shared memory
 // The running maximum is only raised when it grows by more than 2^8, so O is
 // rescaled rarely; the final 1/l uses the same maximum as P, so the result is
-// the exact softmax up to rounding.
+// the exact softmax up to rounding. Where head_dim sits below its 16-column
+// padding (40 -> 48) the row sum l comes from the tensor core: V's first
+// padding column is set to 1 in shared memory (warp 3, after each K/V tile
+// lands), so PV accumulates l = sum_k P[:, k] into O[:, head_dim], in the
+// same fp16 P as the numerator and rescaled with it (level-64 launch 3.11 ->
+// 2.95 ms: 48 packed adds per softmax warp and tile fewer).
 //
 // Roles: warpgroup 0 = warp 0 TMA producer (Q once, K/V tiles into a STAGES
 // ring), warp 1 MMA issuer of query tile 0 and TMEM owner, warp 2 MMA issuer
 // of query tile 1 when each tile has two S buffers (else warp 1 issues both,
-// which measured faster there; warp 3 idle); warpgroups 1 and 2 = softmax of
+// which measured faster there); warp 3 writes V's ones column where the row
+// sums come from the tensor core (else idle); warpgroups 1 and 2 = softmax of
 // query tiles 0 and 1.
 // setmaxnreg moves registers from warpgroup 0 (120 per thread) to the softmax
 // warpgroups (184 per thread); the launch is refused unless the kernel was
@@ -70,10 +76,14 @@ struct Cfg {
   static_assert(BN % 32 == 0 && STAGES >= 2, "tile shape");
   static constexpr uint32_t O_COL = 2 * SB * BN;          // TMEM column of O_0
   static constexpr size_t SMEM = Q_BYTES + STAGES * STAGE_BYTES + 1024 + 512;
+  // head_dim below its 16-column padding: V's first padding column is set to
+  // 1 in shared memory, so PV also accumulates the row sum l of P into
+  // O[:, HD] (the softmax keeps no sums)
+  static constexpr bool ONES = HDP > HD;
   static_assert(2 * SB * BN + 2 * HDP <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   // barriers, TMEM slot, abort flag and segment lengths fit the 512-byte tail
-  static_assert(8 * (18 + 2 * STAGES + 2 * SB) + 8 + 4 * kAttnMaxSegs <= 512, "barrier area");
+  static_assert(8 * (18 + 3 * STAGES + 2 * SB) + 8 + 4 * kAttnMaxSegs <= 512, "barrier area");
 };
 
 constexpr int kThreads = 384;
@@ -101,7 +111,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                                              // one phase for the next-to-last PV (two S buffers)
   uint64_t* o_final = o_full + 2;            // [2 tiles], one phase: the tile's last PV done
   uint64_t* stagger = o_final + 2;           // one phase: tile 0 has reached its first exps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stagger + 1);
+  uint64_t* v_ready = stagger + 1;           // [STAGES]: V's ones column written (ONES)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(v_ready + C::STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // segment lengths, copied once from the parameter space (a constant-cache
   // miss costs several hundred clocks on a warp's critical path)
@@ -143,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       mbar_init(&o_final[i], 1);
     }
     mbar_init(stagger, 128);
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(&v_ready[s], 1);
     for (int sg = 0; sg < n_active; ++sg) seg_len[sg] = p.seg[sg].len;
     *abort_flag = 0;
     fence_barrier_init();
@@ -285,6 +297,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           const bool ahead = jt + 2 < nt_total;
           if (!(ok = wait_p(i, jt))) break;
           if (ahead && !(ok = wait_kv(jt + 2))) break;
+          if (C::ONES) {
+            if (!(ok = mbar_wait(&v_ready[st], (jt / C::STAGES) & 1, abort_flag))) break;
+            tc_fence_after();
+          }
           issue_pv(i, st, b, jt > 0, jt == nt_total - 2);
           if (jt == nt_total - 1) mma_commit(&o_final[i]);
           mma_commit(&kv_empty[st]);
@@ -320,6 +336,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           }
         }
       }
+    }
+    __syncwarp();
+  } else if (C::ONES && warp == 3) {
+    // ------------------------------------------------------------ ones column
+    // V[:, HD] := 1 in each K/V stage once its tile has landed (the TMA
+    // zero-fills the padding columns); 128-byte swizzle: 16-byte unit u of
+    // row r sits at unit u ^ (r & 7)
+    int nt_total = 0;
+    for (int sg = 0; sg < n_active; ++sg) nt_total += (seg_len[sg] + C::BN - 1) / C::BN;
+    constexpr uint32_t kBlk = HD / 64, kUnit = (HD % 64) * 2 / 16, kByte = (HD % 64) * 2 % 16;
+    for (int t = 0; t < nt_total; ++t) {
+      const int st = t % C::STAGES;
+      if (!mbar_wait(&kv_full[st], (t / C::STAGES) & 1, abort_flag)) break;
+      uint8_t* sv = sKV + st * C::STAGE_BYTES + C::K_BYTES + kBlk * C::KV_BLK;
+      for (int r = lane; r < C::BN; r += 32)
+        *reinterpret_cast<__half*>(sv + r * 128 + (((kUnit ^ (r & 7)) << 4) | kByte)) =
+            __float2half(1.0f);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&v_ready[st]);
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -427,14 +463,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 f2_unpack(x, x0, x1);
                 pp = f2_pack(ex2_f32(x0), ex2_f32(x1));
               }
-              accs[e & 3] = f2_add(accs[e & 3], pp);
+              if constexpr (!C::ONES) accs[e & 3] = f2_add(accs[e & 3], pp);
               float p0, p1;
               f2_unpack(pp, p0, p1);
               pk[e] = h2_from(p0, p1);
             }
-            float a0, a1;
-            f2_unpack(f2_add(f2_add(accs[0], accs[1]), f2_add(accs[2], accs[3])), a0, a1);
-            sum += a0 + a1;
+            if constexpr (!C::ONES) {
+              float a0, a1;
+              f2_unpack(f2_add(f2_add(accs[0], accs[1]), f2_add(accs[2], accs[3])), a0, a1);
+              sum += a0 + a1;
+            }
           }
           tmem_st16(s_addr + c / 2, pk);
         }
@@ -449,7 +487,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     // earlier PV (with two S buffers the last two PVs can both be in flight)
     if (ok && jt > 0 && mbar_wait(&o_final[i], 0, abort_flag)) {
       tc_fence_after();
-      const float inv = 1.0f / l_run;
+      float l_fin = l_run;
+      if constexpr (C::ONES) {
+        uint32_t r[16];
+        tmem_ld16(o_addr + HD / 16 * 16, r);
+        tmem_wait_ld();
+        l_fin = __uint_as_float(r[HD % 16]);
+      }
+      const float inv = 1.0f / l_fin;
       const int grow = q_row0 + 128 * i + row;
       const bool store = grow < p.n_q;
       __half* orow = p.out + static_cast<int64_t>(frame) * p.out_fstride +

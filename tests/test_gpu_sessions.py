@@ -167,3 +167,39 @@ def test_batched_sessions_equal_single_streams(P):
     batched.close()
     for s in singles:
         s.close()
+
+
+def test_sessions_host_round_equals_device_round(P):
+    # the host-buffer round with S = 3 (staging sets scaled by S, two sets
+    # alternating) against the device round of an identical context; three
+    # rounds enqueued before one synchronisation
+    sess = _sessions([3.0, 0.5, 3.0])
+    dev_ctx = _ctx(P, sess)
+    host_ctx = _ctx(P, sess)
+    stream = torch.cuda.Stream()
+    rounds = []
+    for r in range(1, 4):
+        inputs = []
+        for z in sess:
+            hidden, noise, eps = z.round_inputs(r)
+            inputs.append((hidden, noise, eps, z.next_motion(r)))
+        rounds.append(inputs)
+    want = [_run_round(dev_ctx, sess, inputs, stream)[0] for inputs in rounds]
+    pin = lambda xs: torch.from_numpy(np.ascontiguousarray(np.stack(xs))).pin_memory()
+    h_args, h_out = [], []
+    for inputs in rounds:
+        h_hidden = [pin([inp[0][li] for inp in inputs]) for li in range(len(LAYERS))]
+        h_args.append((pin([inp[1] for inp in inputs]), pin([inp[3] for inp in inputs]), h_hidden,
+                       pin([inp[2] for inp in inputs])))
+        h_out.append(torch.full((len(sess), 4, 4, H, W), float("nan")).pin_memory())
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for (hn, hm, hh, he), ho in zip(h_args, h_out):
+            host_ctx.round_host(hn, hm, hh, he, ho, stream=stream)
+    stream.synchronize()
+    for r, (w, ho) in enumerate(zip(want, h_out)):
+        assert np.array_equal(ho.numpy(), w), r
+    for zi in range(len(sess)):
+        assert host_ctx.state(session=zi) == dev_ctx.state(session=zi), zi
+    dev_ctx.close()
+    host_ctx.close()
