@@ -71,7 +71,7 @@ def peaks():
 
 def kernel_hash() -> str:
     h = hashlib.sha256()
-    for f in ("attn.cu", "attn.cuh", "ptx.cuh"):
+    for f in ("attn.cu", "attn.cuh", "ptx.cuh", "fastmath.cuh"):
         with open(os.path.join(ROOT, "denoise_step_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
