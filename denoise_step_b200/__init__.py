@@ -401,6 +401,20 @@ class Stream:
         for t in [h_noise, h_motion, h_eps, h_out_frames, *h_hidden]:
             if t.is_cuda or not t.is_contiguous():
                 raise ValueError("round_host takes contiguous host tensors")
+        # the C call copies fixed byte counts from these pointers: check them here
+        c = self.cfg
+        S = max(c.sessions, 1)
+        fe = c.latent_c * c.latent_h * c.latent_w
+        want = [(h_noise, torch.float32, S * 4 * fe), (h_motion, torch.float32, S * 4 * 512),
+                (h_eps, torch.float32, S * 16 * fe), (h_out_frames, torch.float32, S * 4 * fe)]
+        if len(h_hidden) != c.n_layers:
+            raise ValueError(f"round_host: {len(h_hidden)} hidden tensors for {c.n_layers} layers")
+        want += [(h, torch.float16, S * 16 * c.layer_tokens[l] * c.layer_channels[l])
+                 for l, h in enumerate(h_hidden)]
+        for t, dt, n in want:
+            if t.dtype != dt or t.numel() != n:
+                raise ValueError(f"round_host: expected {dt} with {n} elements, got {t.dtype} "
+                                 f"with {t.numel()}")
         hp = _ptr_array(h_hidden) if self.cfg.n_layers else None
         check(lib.pl_stream_round_host(self.handle, _ptr(self._staging), self._staging.numel(),
                                        _ptr(h_noise), _ptr(h_motion), hp, _ptr(h_eps),

@@ -156,3 +156,30 @@ def test_rope_and_lpm_validation():
     assert L.pl_rope_table(None, 10, 64, 10000.0, None) == P.PL_EINVAL
     assert L.pl_rope_table(C.c_void_p(256), 10, 63, 10000.0, None) == P.PL_EINVAL
     assert L.pl_rope_attention_workspace_bytes(0, 10, 1, 64, C.byref(n)) == P.PL_EINVAL
+
+
+def test_round_host_binding_checks_host_tensors():
+    # the binding refuses host tensors of the wrong size or type before any C
+    # call (the C side copies fixed byte counts from the pointers it is given)
+    import torch
+    import denoise_step_b200 as P
+
+    class Fake(P.Stream):
+        def __init__(self, cfg):       # no device workspace, no context
+            self.cfg = cfg
+            self.handle = None
+            self._staging = torch.empty(0, dtype=torch.uint8)
+
+    cfg = P.make_config((8, 8), [(64, 320)])
+    st = Fake(cfg)
+    fe = 4 * 8 * 8
+    ok = dict(h_noise=torch.zeros(4 * fe), h_motion=torch.zeros(4 * 512),
+              h_hidden=[torch.zeros(16 * 64 * 320, dtype=torch.float16)],
+              h_eps=torch.zeros(16 * fe), h_out_frames=torch.zeros(4 * fe))
+    for key, bad in [("h_noise", torch.zeros(4 * fe - 1)),
+                     ("h_eps", torch.zeros(16 * fe, dtype=torch.float64)),
+                     ("h_hidden", [torch.zeros(16 * 64 * 320)]),
+                     ("h_hidden", [])]:
+        args = dict(ok, **{key: bad})
+        with pytest.raises(ValueError):
+            st.round_host(**args)
