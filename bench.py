@@ -46,6 +46,11 @@ def attn_flops_layer(N: int, C: int, kv_entries: int = 5, frames: int = 16) -> f
     return 4.0 * frames * S.HEADS * N * (kv_entries * N) * hd
 
 
+def exp2_level64(N: int = 4096, kv_entries: int = 5, frames: int = 16) -> float:
+    """exp2 evaluations of one 64x64-level attention launch: one per (frame, head, query, key)."""
+    return float(frames * S.HEADS * N * kv_entries * N)
+
+
 def round_attn_flops() -> float:
     return sum(attn_flops_layer(side * side, C) for _, side, C in S.LAYERS)
 
@@ -581,6 +586,15 @@ def run_ours(args, rank, world, local_rank):
             "round_tflops_effective": (round_attn_flops() + round_proj_flops()) * args.steps / elapsed / 1e12 / world,
             "attn_tflops_level64": achieved,
             "attn_frac_fp16_peak": {"measured": achieved / tf_peak, "spec_2250": achieved / 2250.0},
+            # the same launch counted in exp2 evaluations (one per score; at
+            # head_dim 40 the exp2 units, not the tensor pipe, bound it): 11 of
+            # every 16 go to the MUFU (16 per clock per SM), the rest to an
+            # FMA-pipe polynomial
+            "attn_exp2_level64": {
+                "exp2_per_s": exp2_level64() / attn_s,
+                "mufu_exp2_per_s": exp2_level64() * 11 / 16 / attn_s,
+                "mufu_peak_per_s": 16 * 148 * 1.965e9,
+                "mufu_frac": exp2_level64() * 11 / 16 / attn_s / (16 * 148 * 1.965e9)},
             "l2": "per-step inputs (~0.4 GB hidden + bank K/V) exceed the 126 MB L2; no flush",
         },
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
