@@ -375,10 +375,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     // first exps: the warpgroups' exp phases then start out of step and
     // interleave on the MUFU for the first KV tiles instead of coinciding
     // (measured 3% faster over a level-64 launch; in steady state the two
-    // drift back into step).
+    // drift back into step). Only on the 96-key schedule: with 64-key tiles
+    // (head_dim 80) it measured 1.3% slower and with 96-key ones without it
+    // 1% slower.
     int nt_all = 0;
     for (int sg = 0; sg < n_active; ++sg) nt_all += (seg_len[sg] + C::BN - 1) / C::BN;
-    if (C::SB == 2 && i == 1 && n_active > 0) ok = mbar_wait(stagger, 0, abort_flag);
+    if (C::V2 && C::SB == 2 && i == 1 && n_active > 0) ok = mbar_wait(stagger, 0, abort_flag);
     for (int sg = 0; ok && sg < n_active; ++sg) {
       const int len = seg_len[sg];
       const int nt = (len + C::BN - 1) / C::BN;
