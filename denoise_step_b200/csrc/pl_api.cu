@@ -607,15 +607,13 @@ pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_
 pl_status pl_ctx_destroy(pl_ctx* ctx) {
   if (!ctx) return PL_OK;
   drop_graph(ctx);
+  // the staging the copies write belongs to the caller: finish them first
+  if (ctx->copy_stream) cudaStreamSynchronize(ctx->copy_stream);
   for (int b = 0; b < 2; ++b) {
     if (ctx->ev_in[b]) cudaEventDestroy(ctx->ev_in[b]);
     if (ctx->ev_free[b]) cudaEventDestroy(ctx->ev_free[b]);
   }
-  if (ctx->copy_stream) {
-    // the staging the copies write belongs to the caller: finish them first
-    cudaStreamSynchronize(ctx->copy_stream);
-    cudaStreamDestroy(ctx->copy_stream);
-  }
+  if (ctx->copy_stream) cudaStreamDestroy(ctx->copy_stream);
   delete ctx;
   return PL_OK;
 }
