@@ -61,3 +61,28 @@ def test_reference_arm_other_ranks_exit_quietly(capsys):
 def test_job_rate_single():
     import bench
     assert bench.job_rate(1, 20, 0.5) == pytest.approx(40.0)
+
+
+def test_attention_work_units_and_traffic_key(tmp_path, monkeypatch):
+    # the units the roofline figures are built from, and the key that voids a
+    # stored DRAM-traffic figure once any attention source changes
+    import shutil
+
+    import bench
+    assert bench.attn_flops_layer(4096, 320) == 4.0 * 16 * 8 * 4096 * (5 * 4096) * 40
+    assert abs(bench.attn_flops_layer(4096, 320) / 1e12 - 1.718) < 1e-3
+    assert bench.exp2_level64() == 16 * 8 * 4096 * 5 * 4096
+    src = os.path.join(bench.ROOT, "denoise_step_b200", "csrc")
+    dst = tmp_path / "denoise_step_b200" / "csrc"
+    dst.mkdir(parents=True)
+    names = ("attn.cu", "attn.cuh", "ptx.cuh", "fastmath.cuh")
+    for f in names:
+        shutil.copy(os.path.join(src, f), dst / f)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    base = bench.kernel_hash()
+    for f in names:
+        keep = (dst / f).read_bytes()
+        (dst / f).write_bytes(keep + b"\n")
+        assert bench.kernel_hash() != base, f
+        (dst / f).write_bytes(keep)
+    assert bench.kernel_hash() == base
