@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -38,6 +39,14 @@ WORKLOAD = ("full round at 512x512 geometry: 16 reference-attention layers in SD
             "(64x64/C320 x5, 32x32/C640 x5, 16x16/C1280 x5, 8x8/C1280 x1; 8 heads), "
             "KV = own + bank x4, motion x-attn 32x16-d per layer, DDIM on 16x4x64x64, bank check")
 SEED = S.SEEDS["full"]
+L2_NOTE = "per-step inputs (~0.4 GB hidden + bank K/V) exceed the 126 MB L2; no flush"
+
+
+def bench_config(world: int) -> dict:
+    """The `config` both arms print (the same dict, so the two lines name one workload)."""
+    return {"workload": WORKLOAD,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": L2_NOTE}
 
 
 def attn_flops_layer(N: int, C: int, kv_entries: int = 5, frames: int = 16) -> float:
@@ -237,7 +246,7 @@ def run_reference(args, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": per_round * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "frames_per_s": 4 * value},
+        "config": bench_config(args.gpus), "frames_per_s": 4 * value,
         "cpu_baseline": {"value": value, "unit": "rounds/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "rounds/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -422,6 +431,104 @@ def pose_front(torch, P, stream, hbm_peak):
     return out
 
 
+def tiny_round(torch, P, stream):
+    """C1: the round at the tiny geometry (one 8x8-token level, C 1280, 8 heads of
+    160, KV = own + bank x1, motion x-attn, DDIM on 16x4x8x8, bank check of 4
+    new embeddings) through pl_stream_round with device-resident inputs, and the
+    context-free bank check of 4 N(0,4) queries against 8 stored N(0,4) vectors;
+    microseconds per call by CUDA events over back-to-back calls."""
+    seed, H, W, N, C = S.SEEDS["tiny"], 8, 8, 64, 1280
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    w = S.layer_weights(seed, "m", C, np.float16)
+    pw = {"w_qkv": dev(np.concatenate([w["wq"], w["wk"], w["wv"]], 1)), "w_o": dev(w["wo"]),
+          "m_q": dev(w["mq"]), "m_kv": dev(np.concatenate([w["mk"], w["mv"]], 1)),
+          "m_o": dev(w["mo"])}
+    st = P.Stream(P.make_config((H, W), [(N, C)]))
+    ref_m = S.normal(seed, "walk/e0", (512,), 1.0, np.float32)
+    st.bank_init([pw], [dev(S.bank_features(seed, "m", 0, N, C))], None, dev(ref_m),
+                 dev(S.normal(seed, "drive0", (512,), 1.0, np.float32)),
+                 dev(S.normal(seed, "ref_latent", (4, H, W), 1.0, np.float32)),
+                 dev(S.normal(seed, "prefill_eps", (12, 4, H, W), 1.0, np.float32)), stream=stream)
+    hidden = [dev(S.layer_hidden(seed, "m", 1, 16, N, C))]
+    noise = dev(S.normal(seed, "noise1", (4, 4, H, W), 1.0, np.float32))
+    mot = dev((ref_m[None] + S.normal(seed, "walk/step1", (4, 512), 3.0).cumsum(0)).astype(np.float32))
+    eps = dev(S.normal(seed, "eps1", (16, 4, H, W), 1.0, np.float32))
+    out = torch.empty((4, 4, H, W), dtype=torch.float32, device="cuda")
+    flags = torch.zeros(4, dtype=torch.uint8, device="cuda")
+    reps = 200
+    t = _event_time(torch, lambda: st.round(noise, mot, hidden, eps, out, flags, None,
+                                            stream=stream), reps, stream)
+    st.close()
+    bank = dev(S.normal(seed, "bank8", (8, 512), 2.0, np.float32))
+    qs = dev(S.normal(seed, "bankq", (4, 512), 2.0, np.float32))
+    cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+    app = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def check():
+        cnt.fill_(8)
+        app.fill_(0)
+        P.motion_bank_check(bank, cnt, app, qs, 17.0, 3, stream=stream)
+
+    tb = _event_time(torch, check, reps, stream)
+    return {"us_per_round": t * 1e6, "rounds_per_s": 1.0 / t, "frames_per_s": 4.0 / t,
+            "bank_check_8x512_us": tb * 1e6,
+            "note": "bank check timed with two 4-byte fills of its counters per call"}
+
+
+def level64_bank1(torch, P, stream, tf_peak):
+    """C2: one 64x64 level (16 frames x 4096 tokens, C 320, 8 heads of 40, KV =
+    own + bank x1 = 8192) through pl_ref_attention (QKV projection, bank K/V
+    projection, attention core, O projection), the attention core alone at that
+    shape, and the pile DDIM step on 16x4x64x64 (ring push + step)."""
+    seed, F, N, C, heads = S.SEEDS["level64"], 16, 4096, 320, 8
+    hd = C // heads
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    w = S.layer_weights(seed, "L", C, np.float16)
+    w_qkv = dev(np.concatenate([w["wq"], w["wk"], w["wv"]], 1))
+    w_o = dev(w["wo"])
+    h = dev(S.normal(seed, "hidden", (F, N, C), 1.0, np.float16))
+    bank = [dev(S.bank_features(seed, "L", 0, N, C))]
+    out = torch.empty_like(h)
+    need = P.sz()
+    P.check(P.lib.pl_ref_attention_workspace_bytes(F, N, C, 1, P.C.byref(need)), "ws")
+    ws = torch.empty(need.value, dtype=torch.uint8, device="cuda")
+    t_layer = _event_time(torch, lambda: P.ref_attention(h, w_qkv, w_o, bank, heads, out=out,
+                                                         workspace=ws, stream=stream), 10, stream)
+    core = 4.0 * F * heads * N * (2 * N) * hd
+    proj = 2.0 * F * N * C * (3 * C) + 2.0 * F * N * C * C + 2.0 * N * C * (2 * C)
+    # attention core alone on the layer's own Q/K/V (the workspace's first 3 F N C halves)
+    qkv = ws[: 2 * 3 * F * N * C].view(torch.float16).view(F, N, 3 * C)
+    bkv = torch.randn((N, 2 * C), device="cuda", dtype=torch.float16,
+                      generator=torch.Generator(device="cuda").manual_seed(seed))
+    segs = [(qkv[:, :, C:2 * C], qkv[:, :, 2 * C:]), (bkv[:, :C], bkv[:, C:])]
+    o2 = torch.empty((F, N, C), device="cuda", dtype=torch.float16)
+    t_core = _event_time(torch, lambda: P.segment_attention(qkv[:, :, :C], segs, heads, hd, out=o2,
+                                                            stream=stream), 10, stream)
+    # pile DDIM step at the configuration size
+    st = P.Stream(P.make_config((64, 64), []))
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    mkf = lambda *sh: torch.randn(sh, device="cuda", generator=g)
+    st.bank_init([], [], None, mkf(512), mkf(512), mkf(4, 64, 64), mkf(12, 4, 64, 64), stream=stream)
+    noise, mot, eps = mkf(4, 4, 64, 64), mkf(4, 512), mkf(16, 4, 64, 64)
+    xo = torch.empty((4, 4, 64, 64), device="cuda")
+
+    def ddim_round():
+        st.ring_push(noise, mot, stream=stream)
+        st.ddim_step(eps, xo, stream=stream)
+
+    t_ddim = _event_time(torch, ddim_round, 50, stream)
+    st.close()
+    fe = 4 * 64 * 64
+    byts = 4.0 * fe * (8 + 48)
+    return {"layer_ms": t_layer * 1e3, "layer_tflop": (core + proj) / 1e12,
+            "layer_tflops": (core + proj) / t_layer / 1e12,
+            "layer_frac_of_peak": (core + proj) / t_layer / 1e12 / tf_peak,
+            "core_ms": t_core * 1e3, "core_tflops": core / t_core / 1e12,
+            "core_frac_of_peak": core / t_core / 1e12 / tf_peak,
+            "ddim_push_step_us": t_ddim * 1e6, "ddim_gbs": byts / t_ddim / 1e9,
+            "ddim_note": "3.2 MB step, L2-resident and latency-bound at this size"}
+
+
 def secondary_measurements(torch, P, stream, hbm_peak):
     """The other workloads' kernels, timed live (CUDA events on their stream):
     the PR-Sink block (4096 tokens x 40 heads x 128, KV own + sink + retrieved
@@ -517,8 +624,8 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize()
 
-    clk_path = os.path.join(ROOT, "gpurun_out", f"bench_clocks_r{rank}.csv")
-    os.makedirs(os.path.dirname(clk_path), exist_ok=True)
+    clk_dir = tempfile.mkdtemp(prefix="pl_bench_clocks_")
+    clk_path = os.path.join(clk_dir, f"clocks_r{rank}.csv")
     proc, fh = clocks_sampler(local_rank, clk_path)
     time.sleep(0.3)
     barrier()
@@ -578,9 +685,9 @@ def run_ours(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
-        "config": {
-            "workload": WORKLOAD, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "frames_per_s": 4 * value,
+        "config": bench_config(world),
+        "frames_per_s": 4 * value,
+        "detail": {
             "round_attn_tflop": round_attn_flops() / 1e12,
             "round_proj_tflop": round_proj_flops() / 1e12,
             "round_tflops_effective": (round_attn_flops() + round_proj_flops()) * args.steps / elapsed / 1e12 / world,
@@ -595,7 +702,6 @@ def run_ours(args, rank, world, local_rank):
                 "mufu_exp2_per_s": exp2_level64() * 11 / 16 / attn_s,
                 "mufu_peak_per_s": 16 * 148 * 1.965e9,
                 "mufu_frac": exp2_level64() * 11 / 16 / attn_s / (16 * 148 * 1.965e9)},
-            "l2": "per-step inputs (~0.4 GB hidden + bank K/V) exceed the 126 MB L2; no flush",
         },
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
                      "frac": achieved / tf_peak, "traffic": ncu_traffic(),
@@ -610,12 +716,19 @@ def run_ours(args, rank, world, local_rank):
     }
     if rank == 0 and not args.no_secondary:
         sec = secondary_measurements(torch, P, stream, hbm_peak)
+        sec["c1_tiny_round"] = tiny_round(torch, P, stream)
+        sec["c2_level64_bank1"] = level64_bank1(torch, P, stream, tf_peak)
         sec["sessions_4"] = sessions_round(torch, P, wl, stream, 4, elapsed / args.steps * 1e3)
         sec["pr_sink_cache_step"] = sink_stream_step(torch, P, stream)
         sec["lpm_window_step"] = lpm_window_step(torch, P, stream)
         sec["pose_front_512"] = pose_front(torch, P, stream, hbm_peak)
-        line["config"]["secondary"] = sec
+        line["detail"]["secondary"] = sec
     clk = clocks_summary(clk_path)
+    try:
+        os.remove(clk_path)
+        os.rmdir(clk_dir)
+    except OSError:
+        pass
     if clk is not None:
         line["clocks"] = clk
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -15,6 +15,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libpl.so")
 
 PL_OK, PL_EINVAL, PL_ESTATE, PL_ENOMEM, PL_ECUDA, PL_ETIMEOUT, PL_EDEVICE, PL_EUNSUPPORTED = range(8)
+PL_TEST_NO_KV, PL_TEST_BAD_BOX = 1, 2
 MAX_LAYERS = 16
 
 
@@ -82,6 +83,9 @@ _SIGS = {
     "pl_gemm_f16": (i32, [vp, i64, vp, i64, vp, i64, i32, i32, i32, vp]),
     "pl_segment_attention": (i32, [vp, i64, i64, C.POINTER(KVSegment), i32, i32, i32, i32, i32,
                                    vp, i64, i64, vp]),
+    "pl_test_segment_attention_fault": (i32, [vp, i64, i64, C.POINTER(KVSegment), i32, i32, i32,
+                                              i32, i32, vp, i64, i64, i32, C.c_uint32, vp]),
+    "pl_get_call_status": (i32, [vp]),
     "pl_pr_sink_attention": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, C.POINTER(vp),
                                    C.POINTER(vp), i32, i32, i32, i32, vp, vp, vp, vp]),
     "pl_ref_attention_workspace_bytes": (i32, [i32, i32, i32, i32, C.POINTER(sz)]),
@@ -183,6 +187,34 @@ def gemm(a, b, out=None, stream=None):
     return out
 
 
+def _segments(segments):
+    segs = (KVSegment * len(segments))()
+    for i, (k, v) in enumerate(segments):
+        if k.dim() == 3:
+            segs[i] = KVSegment(_ptr(k), _ptr(v), k.shape[1], k.stride(1), k.stride(0))
+        else:
+            segs[i] = KVSegment(_ptr(k), _ptr(v), k.shape[0], k.stride(0), 0)
+    return segs
+
+
+def call_status(stream=None) -> int:
+    """Synchronise `stream` and read (and clear) the device status word of the
+    context-free calls: PL_OK, PL_ETIMEOUT or PL_EDEVICE."""
+    return lib.pl_get_call_status(_stream(stream))
+
+
+def segment_attention_fault(q, segments, heads, head_dim, mode, wait_us, out, stream=None):
+    """pl_test_segment_attention_fault: segment attention with a planted device-side
+    failure (PL_TEST_NO_KV: the bounded waits run out; PL_TEST_BAD_BOX: the kernel
+    refuses its box). Returns the launch status; read the outcome with call_status()."""
+    F, Nq = q.shape[0], q.shape[1]
+    segs = _segments(segments)
+    return lib.pl_test_segment_attention_fault(_ptr(q), q.stride(1), q.stride(0), segs,
+                                               len(segments), F, Nq, heads, head_dim, _ptr(out),
+                                               out.stride(1), out.stride(0), int(mode),
+                                               int(wait_us), _stream(stream))
+
+
 def segment_attention(q, segments, heads, head_dim, out=None, stream=None):
     """Attention of q [F, Nq, ld] over KV segments (k, v, frame_shared) without concatenation.
 
@@ -190,12 +222,7 @@ def segment_attention(q, segments, heads, head_dim, out=None, stream=None):
     """
     import torch
     F, Nq = q.shape[0], q.shape[1]
-    segs = (KVSegment * len(segments))()
-    for i, (k, v) in enumerate(segments):
-        if k.dim() == 3:
-            segs[i] = KVSegment(_ptr(k), _ptr(v), k.shape[1], k.stride(1), k.stride(0))
-        else:
-            segs[i] = KVSegment(_ptr(k), _ptr(v), k.shape[0], k.stride(0), 0)
+    segs = _segments(segments)
     if out is None:
         out = torch.empty((F, Nq, heads * head_dim), dtype=torch.float16, device=q.device)
     check(lib.pl_segment_attention(_ptr(q), q.stride(1), q.stride(0), segs, len(segments), F, Nq,

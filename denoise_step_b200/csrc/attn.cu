@@ -42,8 +42,10 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <mutex>
 
 #include "attn.cuh"
+#include "devinit.cuh"
 #include "fastmath.cuh"
 #include "ptx.cuh"
 #include "tmap.cuh"
@@ -83,7 +85,7 @@ struct Cfg {
   static_assert(2 * SB * BN + 2 * HDP <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   // barriers, TMEM slot, abort flag and segment lengths fit the 512-byte tail
-  static_assert(8 * (18 + 3 * STAGES + 2 * SB) + 8 + 4 * kAttnMaxSegs <= 512, "barrier area");
+  static_assert(8 * (20 + 3 * STAGES + 2 * SB) + 8 + 4 * kAttnMaxSegs <= 512, "barrier area");
 };
 
 constexpr int kThreads = 384;
@@ -112,7 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   uint64_t* o_final = o_full + 2;            // [2 tiles], one phase: the tile's last PV done
   uint64_t* stagger = o_final + 2;           // one phase: tile 0 has reached its first exps
   uint64_t* v_ready = stagger + 1;           // [STAGES]: V's ones column written (ONES)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(v_ready + C::STAGES);
+  uint64_t* drain = v_ready + C::STAGES;     // [2 issuers]: their MMAs done (after an abort)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // segment lengths, copied once from the parameter space (a constant-cache
   // miss costs several hundred clocks on a warp's critical path)
@@ -123,6 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   const int q_row0 = blockIdx.x * 256;
   const int head = blockIdx.y;
   const int frame = blockIdx.z;
+  const uint64_t wl = p.wait_ns;   // limit of every bounded wait
 
   // the K/V boxes the host encoded must match this kernel's key tile, or the
   // TMA writes would not fit the stage buffers: refuse to run
@@ -155,6 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     }
     mbar_init(stagger, 128);
     for (int s = 0; s < C::STAGES; ++s) mbar_init(&v_ready[s], 1);
+    for (int w = 0; w < 2; ++w) mbar_init(&drain[w], 1);
     for (int sg = 0; sg < n_active; ++sg) seg_len[sg] = p.seg[sg].len;
     *abort_flag = 0;
     fence_barrier_init();
@@ -183,7 +188,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                       q_row0 + 128 * i, frame);
       int stage = 0;
       uint32_t phase = 0;
-      for (int sg = 0; sg < n_active && !*abort_flag; ++sg) {
+      int issued = 0;   // K/V tiles whose copies were started
+      // planted failure (test hook): no K/V tile is loaded, so the consumers'
+      // bounded waits run out with no copy in flight
+      const int n_load = p.test_mode == kTestNoKV ? 0 : n_active;
+      for (int sg = 0; sg < n_load && !*abort_flag; ++sg) {
         const AttnSeg& seg = p.seg[sg];
         int fr = seg.per_frame ? frame : (seg.frame_div > 0 ? frame / seg.frame_div : 0);
         if (seg.block_sel != nullptr) {
@@ -195,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
         const int nt = (seg.len + C::BN - 1) / C::BN;
         for (int lt = 0; lt < nt; ++lt) {
-          if (!mbar_wait(&kv_empty[stage], phase ^ 1, abort_flag)) break;
+          if (!mbar_wait(&kv_empty[stage], phase ^ 1, abort_flag, wl)) break;
           uint8_t* sk = sKV + stage * C::STAGE_BYTES;
           uint8_t* sv = sk + C::K_BYTES;
           mbar_expect_tx(&kv_full[stage], C::STAGE_BYTES);
@@ -205,11 +214,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 #pragma unroll
           for (int b = 0; b < C::NBLK; ++b)
             tma_load_4d(sv + b * C::KV_BLK, &seg.v, &kv_full[stage], 64 * b, head, lt * C::BN, fr);
+          ++issued;
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
+      }
+      if (*abort_flag) {
+        // let the copies still in flight (at most the last STAGES tiles and
+        // Q) land before the CTA's shared memory can go to another CTA
+        mbar_wait_drain(q_full, 0, wl);
+        for (int t = issued > C::STAGES ? issued - C::STAGES : 0; t < issued; ++t)
+          mbar_wait_drain(&kv_full[t % C::STAGES], (t / C::STAGES) & 1, wl);
       }
     }
     __syncwarp();
@@ -247,11 +264,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         if (commit_o) mma_commit(&o_full[i]);
       };
       auto wait_p = [&](int i, int jt) {
-        const bool r = mbar_wait(&p_full[i * 2 + (jt & 1)], (jt >> 1) & 1, abort_flag);
+        const bool r = mbar_wait(&p_full[i * 2 + (jt & 1)], (jt >> 1) & 1, abort_flag, wl);
         tc_fence_after();
         return r;
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag);
+      bool ok = mbar_wait(q_full, 0, abort_flag, wl);
       tc_fence_after();
       // the MMA side only needs the total tile count (the tiles' segments
       // matter to the producer and the softmax)
@@ -283,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         const int i = warp - 1;
         auto stage_of = [](int t) { return t % C::STAGES; };
         auto wait_kv = [&](int t) {
-          const bool r = mbar_wait(&kv_full[stage_of(t)], (t / C::STAGES) & 1, abort_flag);
+          const bool r = mbar_wait(&kv_full[stage_of(t)], (t / C::STAGES) & 1, abort_flag, wl);
           tc_fence_after();
           return r;
         };
@@ -298,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           if (!(ok = wait_p(i, jt))) break;
           if (ahead && !(ok = wait_kv(jt + 2))) break;
           if (C::ONES) {
-            if (!(ok = mbar_wait(&v_ready[st], (jt / C::STAGES) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait(&v_ready[st], (jt / C::STAGES) & 1, abort_flag, wl))) break;
             tc_fence_after();
           }
           issue_pv(i, st, b, jt > 0, jt == nt_total - 2);
@@ -310,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         int prev_stage = 0;
         int jt = 0;
         for (; ok && jt < nt_total; ++jt) {
-          if (!(ok = mbar_wait(&kv_full[stage], phase, abort_flag))) break;
+          if (!(ok = mbar_wait(&kv_full[stage], phase, abort_flag, wl))) break;
           tc_fence_after();
           // one S buffer per tile: PV(jt - 1) must be issued before S(jt)
           // overwrites the P it reads (the tensor pipe runs them in order)
@@ -336,6 +353,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           }
         }
       }
+      if (*abort_flag) {
+        // the MMAs this thread queued must finish before TMEM is freed
+        mma_commit(&drain[warp - 1]);
+        mbar_wait_drain(&drain[warp - 1], 0, wl);
+      }
     }
     __syncwarp();
   } else if (C::ONES && warp == 3) {
@@ -348,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     constexpr uint32_t kBlk = HD / 64, kUnit = (HD % 64) * 2 / 16, kByte = (HD % 64) * 2 % 16;
     for (int t = 0; t < nt_total; ++t) {
       const int st = t % C::STAGES;
-      if (!mbar_wait(&kv_full[st], (t / C::STAGES) & 1, abort_flag)) break;
+      if (!mbar_wait(&kv_full[st], (t / C::STAGES) & 1, abort_flag, wl)) break;
       uint8_t* sv = sKV + st * C::STAGE_BYTES + C::K_BYTES + kBlk * C::KV_BLK;
       for (int r = lane; r < C::BN; r += 32)
         *reinterpret_cast<__half*>(sv + r * 128 + (((kUnit ^ (r & 7)) << 4) | kByte)) =
@@ -380,14 +402,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     // 1% slower.
     int nt_all = 0;
     for (int sg = 0; sg < n_active; ++sg) nt_all += (seg_len[sg] + C::BN - 1) / C::BN;
-    if (C::V2 && C::SB == 2 && i == 1 && n_active > 0) ok = mbar_wait(stagger, 0, abort_flag);
+    if (C::V2 && C::SB == 2 && i == 1 && n_active > 0) ok = mbar_wait(stagger, 0, abort_flag, wl);
     for (int sg = 0; ok && sg < n_active; ++sg) {
       const int len = seg_len[sg];
       const int nt = (len + C::BN - 1) / C::BN;
       for (int lt = 0; lt < nt; ++lt) {
         const int b = C::SB == 2 ? (jt & 1) : 0;
         const uint32_t use = C::SB == 2 ? static_cast<uint32_t>(jt >> 1) : static_cast<uint32_t>(jt);
-        if (!(ok = mbar_wait(&s_full[i * C::SB + b], use & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(&s_full[i * C::SB + b], use & 1, abort_flag, wl))) break;
         tc_fence_after();
         const uint32_t s_addr = tmem + lane_off + s_col(i, b);
         float s[C::BN];
@@ -427,10 +449,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           // own one-shot phase on o_full
           if constexpr (C::SB == 2) {
             const bool via_s = jt + 1 < nt_all;
-            ok = via_s ? mbar_wait(&s_full[i * C::SB + ((jt + 1) & 1)], ((jt + 1) >> 1) & 1, abort_flag)
-                       : mbar_wait(&o_full[i], 0, abort_flag);
+            ok = via_s ? mbar_wait(&s_full[i * C::SB + ((jt + 1) & 1)], ((jt + 1) >> 1) & 1, abort_flag, wl)
+                       : mbar_wait(&o_full[i], 0, abort_flag, wl);
           } else {
-            ok = mbar_wait(&o_full[i], (jt - 1) & 1, abort_flag);
+            ok = mbar_wait(&o_full[i], (jt - 1) & 1, abort_flag, wl);
           }
           if (!ok) break;
           tc_fence_after();
@@ -487,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     }
     // o_final has a single phase, so this wait cannot be satisfied by an
     // earlier PV (with two S buffers the last two PVs can both be in flight)
-    if (ok && jt > 0 && mbar_wait(&o_final[i], 0, abort_flag)) {
+    if (ok && jt > 0 && mbar_wait(&o_final[i], 0, abort_flag, wl)) {
       tc_fence_after();
       float l_fin = l_run;
       if constexpr (C::ONES) {
@@ -645,15 +667,22 @@ int attn_make_params(AttnParams* p, const void* q, int64_t ldq, int64_t q_fstrid
   p->scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
   p->box_rows = bn_i;
   p->status = nullptr;
+  p->wait_ns = kWaitLimitNs;
+  p->test_mode = 0;
   return 0;
 }
 
 int attn_init() {
-  static int done = 0;
-  if (!done) {
+  // kernel attributes are per device: set them once on each device used
+  static std::mutex mu;
+  static bool done[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return 4;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
     if (set_attr<40>() || set_attr<64>() || set_attr<80>() || set_attr<128>() || set_attr<160>())
       return 4;
-    done = 1;
+    done[dev] = true;
   }
   return 0;
 }

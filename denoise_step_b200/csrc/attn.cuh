@@ -34,7 +34,13 @@ struct AttnParams {
   float scale_log2;            // log2(e) / sqrt(head_dim)
   int box_rows;                // K/V tensor-map box rows; must equal the kernel's key tile
   uint32_t* status;
+  uint64_t wait_ns;            // limit of each bounded mbarrier wait (ns)
+  int test_mode;               // 0, or kTestNoKV (a planted failure for tests)
 };
+
+// Test hook: the producer loads Q but no K/V tile, so the MMA issuers'
+// bounded waits run out (nothing is in flight when they do).
+constexpr int kTestNoKV = 1;
 
 struct AttnSegHost {
   const void* k;

@@ -3,7 +3,7 @@
 Method: weighted least squares on 4096 Chebyshev nodes, minimising the relative
 error of p(f) against 2^f (a near-minimax fit). Max relative error 7.7e-5,
 below the fp16 rounding of the probabilities (4.9e-4). Prints the fp32 values
-hard-coded in attn.cu.
+written into exp2_poly2() in fastmath.cuh (highest power first there).
 """
 import numpy as np
 

@@ -42,6 +42,9 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 // 2^x for a pair on the FMA pipe: n = nearest integer (1.5 * 2^23 shifter),
 // f = x - n in [-0.5, 0.5], 2^f by a degree-3 polynomial, 2^n added into the
 // exponent field. x is clamped to >= -126 so 2^n stays a normal number.
+// The cubic is a weighted least-squares fit of 2^f on 4096 Chebyshev nodes of
+// [-0.5, 0.5] (relative error minimised; max 7.7e-5, below the 4.9e-4 of the
+// fp16 rounding that P gets next); exp2_poly.py beside this file prints it.
 __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
   float x0, x1;
   f2_unpack(x, x0, x1);

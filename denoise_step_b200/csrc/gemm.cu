@@ -13,6 +13,9 @@
 //               out by a TMA tile store (two chunks in flight per warp)
 #include <cuda_runtime.h>
 
+#include <mutex>
+
+#include "devinit.cuh"
 #include "gemm.cuh"
 #include "ptx.cuh"
 #include "tmap.cuh"
@@ -59,7 +62,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* drain = acc_empty + 2;      // the issuer's MMAs done (after an abort)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -74,6 +78,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -91,6 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
       }
       int stage = 0;
       uint32_t phase = 0;
+      int issued = 0;   // stages whose copies were started
       for (int t = blockIdx.x; t < p.total_tiles && !*abort_flag; t += gridDim.x) {
         TileCoord tc;
         if (!decode_tile(p, t, tc)) continue;
@@ -98,6 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
         const int nk = (pr.K + kGemmBK - 1) / kGemmBK;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+          ++issued;
           uint8_t* sa = smem + stage * kStageBytes;
           uint8_t* sb = sa + kABytes;
           mbar_expect_tx(&full[stage], kStageBytes);
@@ -110,6 +117,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
             phase ^= 1;
           }
         }
+      }
+      if (*abort_flag) {
+        // let the copies still in flight land before the CTA's shared memory
+        // can go to another CTA
+        for (int u = issued > kStages ? issued - kStages : 0; u < issued; ++u)
+          mbar_wait_drain(&full[u % kStages], (u / kStages) & 1);
       }
     }
     __syncwarp();
@@ -162,6 +175,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
         }
         mma_commit(&acc_full[buf]);
         ++acc_i;
+      }
+      if (*abort_flag) {
+        // the MMAs this thread queued must finish before TMEM is freed
+        mma_commit(drain);
+        mbar_wait_drain(drain, 0);
       }
     }
     __syncwarp();
@@ -277,12 +295,17 @@ int gemm_make_problem(GemmProblem* p, const void* a, int64_t lda, const void* b,
 }
 
 int gemm_init() {
-  static int done = 0;
-  if (!done) {
+  // the shared-memory attribute is per device: set it once on each device used
+  static std::mutex mu;
+  static bool done[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return 4;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
     if (cudaFuncSetAttribute(gemm_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes)) != cudaSuccess)
       return 4;
-    done = 1;
+    done[dev] = true;
   }
   return 0;
 }

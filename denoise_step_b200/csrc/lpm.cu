@@ -21,6 +21,7 @@
 
 #include "../../include/pl.h"
 #include "attn.cuh"
+#include "devinit.cuh"
 
 namespace {
 
@@ -245,6 +246,7 @@ pl_status pl_rope_attention(const void* q, int64_t ldq, int q_pos0, const pl_kv_
                                       n_q, heads, head_dim, out, ldo,
                                       static_cast<int64_t>(n_q) * ldo);
   if (mr) return mr == 1 ? PL_EINVAL : PL_ECUDA;
+  p.status = pl::call_status_word();
   return status_of(pl::attn_launch(p, head_dim, st));
 }
 

@@ -23,7 +23,9 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_ptr[kMaxDevices] = {};
 
-// Device address of g_scratch on the current device, looked up once per device.
+// Device address of g_scratch on the current device, looked up once per device
+// and kept: a cudaDeviceReset between calls would leave it stale (pl.h says
+// none may come between calls).
 pl_status scratch_for_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PL_ECUDA;

@@ -5,10 +5,12 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "../../include/pl.h"
 #include "attn.cuh"
+#include "devinit.cuh"
 #include "gemm.cuh"
 #include "misc.cuh"
 #include "ptx.cuh"
@@ -24,16 +26,7 @@ constexpr int kMaxSessions = 8;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-  }
-  return n;
-}
+int num_sms() { return pl::device_sms(); }
 
 bool head_dim_supported(int hd) {
   return hd == 40 || hd == 64 || hd == 80 || hd == 128 || hd == 160;
@@ -45,7 +38,52 @@ pl_status gemm_status(int r) {
   return r == 0 ? PL_OK : r == 1 ? PL_EINVAL : r == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
 }
 
+// Status word of the calls made without a context (one per device that uses
+// the library): kernels OR their device-side problems into it, and
+// pl_get_call_status() reads and clears it.
+static __device__ uint32_t g_call_status;
+
+std::mutex g_dev_mu;
+uint32_t* g_call_status_ptr[pl::kMaxDevices] = {};
+int g_sms[pl::kMaxDevices] = {};
+
 }  // namespace
+
+namespace pl {
+
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+uint32_t* call_status_word() {
+  const int dev = current_device();
+  if (dev < 0) return nullptr;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  if (!g_call_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_call_status) != cudaSuccess) return nullptr;
+    g_call_status_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  return g_call_status_ptr[dev];
+}
+
+int device_sms() {
+  const int dev = current_device();
+  if (dev < 0) return 148;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  if (g_sms[dev] <= 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sms[dev] = n;
+  }
+  return g_sms[dev];
+}
+
+}  // namespace pl
+
 
 // ====================================================================== context
 
@@ -361,7 +399,8 @@ int pl_abi_version(void) { return 1; }
 pl_status pl_gemm_f16(const void* a, int64_t lda, const void* b, int64_t ldb, void* c,
                       int64_t ldc, int M, int N, int K, void* stream) {
   if (!a || !b || !c) return PL_EINVAL;
-  return single_gemm(a, lda, b, ldb, c, ldc, M, N, K, nullptr, static_cast<cudaStream_t>(stream));
+  return single_gemm(a, lda, b, ldb, c, ldc, M, N, K, pl::call_status_word(),
+                     static_cast<cudaStream_t>(stream));
 }
 
 pl_status pl_segment_attention(const void* q, int64_t ldq, int64_t q_frame_stride,
@@ -381,6 +420,40 @@ pl_status pl_segment_attention(const void* q, int64_t ldq, int64_t q_frame_strid
   const int r = pl::attn_make_params(&p, q, ldq, q_frame_stride, hs, n_segs, frames, n_q, heads,
                                      head_dim, out, ldo, out_frame_stride);
   if (r) return r == 1 ? PL_EINVAL : PL_ECUDA;
+  p.status = pl::call_status_word();
+  const int lr = pl::attn_launch(p, head_dim, static_cast<cudaStream_t>(stream));
+  return lr == 0 ? PL_OK : lr == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
+}
+
+pl_status pl_test_segment_attention_fault(const void* q, int64_t ldq, int64_t q_frame_stride,
+                                         const pl_kv_segment* segs, int n_segs, int frames,
+                                         int n_q, int heads, int head_dim, void* out,
+                                         int64_t ldo, int64_t out_frame_stride, int mode,
+                                         uint32_t wait_us, void* stream) {
+  if (!q || !segs || !out) return PL_EINVAL;
+  if (mode != PL_TEST_NO_KV && mode != PL_TEST_BAD_BOX) return PL_EINVAL;
+  if (wait_us < 1 || wait_us > 2000000) return PL_EINVAL;
+  if (n_segs < 1 || n_segs > pl::kAttnMaxSegs) return PL_EINVAL;
+  if (!head_dim_supported(head_dim)) return PL_EUNSUPPORTED;
+  if (frames > 65535 || heads > 65535) return PL_EINVAL;
+  AttnSegHost hs[pl::kAttnMaxSegs];
+  for (int i = 0; i < n_segs; ++i) {
+    if (!segs[i].k || !segs[i].v) return PL_EINVAL;
+    hs[i] = {segs[i].k, segs[i].v, segs[i].len, segs[i].ld, segs[i].frame_stride};
+  }
+  AttnParams p;
+  const int r = pl::attn_make_params(&p, q, ldq, q_frame_stride, hs, n_segs, frames, n_q, heads,
+                                     head_dim, out, ldo, out_frame_stride);
+  if (r) return r == 1 ? PL_EINVAL : PL_ECUDA;
+  p.status = pl::call_status_word();
+  p.wait_ns = static_cast<uint64_t>(wait_us) * 1000ull;
+  if (mode == PL_TEST_NO_KV) {
+    p.test_mode = pl::kTestNoKV;
+  } else {
+    // the tensor maps stay as encoded; only the count the kernel checks
+    // against its key tile is off, so it returns before any copy
+    p.box_rows += 16;
+  }
   const int lr = pl::attn_launch(p, head_dim, static_cast<cudaStream_t>(stream));
   return lr == 0 ? PL_OK : lr == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
 }
@@ -417,6 +490,7 @@ pl_status pl_pr_sink_attention(const void* q, const void* k_own, const void* v_o
   const int mr = pl::attn_make_params(&p, q, ld, static_cast<int64_t>(n) * ld, segs, ns, 1, n,
                                       heads, head_dim, out, ld, static_cast<int64_t>(n) * ld);
   if (mr) return mr == 1 ? PL_EINVAL : PL_ECUDA;
+  p.status = pl::call_status_word();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   pl_status r = from_cuda(pl::launch_nearest(pose_store, n_pool, pose_dim, pose_query, retrieved,
                                              retrieved_d2, s));
@@ -454,8 +528,10 @@ pl_status pl_ref_attention(const void* hidden, const void* w_qkv, const void* w_
                                           align_up(2 * 3 * fnc));
   __half* o = reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(bkv) +
                                         align_up(2 * static_cast<size_t>(n_bank) * n * 2 * c));
+  uint32_t* status = pl::call_status_word();
   GemmParams gp;
   std::memset(&gp, 0, sizeof(gp));
+  gp.status = status;
   int r = pl::gemm_make_problem(&gp.prob[0], hidden, c, w_qkv, 3 * c, qkv, 3 * c, frames * n,
                                 3 * c, c, nullptr);
   if (r) return gemm_status(r);
@@ -480,9 +556,10 @@ pl_status pl_ref_attention(const void* hidden, const void* w_qkv, const void* w_
   r = pl::attn_make_params(&ap, qkv, 3ll * c, static_cast<int64_t>(n) * 3 * c, segs, 1 + n_bank,
                            frames, n, heads, hd, o, c, static_cast<int64_t>(n) * c);
   if (r) return r == 1 ? PL_EINVAL : PL_ECUDA;
+  ap.status = status;
   r = pl::attn_launch(ap, hd, s);
   if (r) return r == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
-  return single_gemm(o, c, w_o, c, out, c, frames * n, c, c, nullptr, s);
+  return single_gemm(o, c, w_o, c, out, c, frames * n, c, c, status, s);
 }
 
 pl_status pl_motion_xattn_workspace_bytes(int frames, int n, int c, size_t* bytes) {
@@ -511,14 +588,15 @@ pl_status pl_motion_xattn(const void* x, const float* motion, const void* m_q, c
   float* qm = reinterpret_cast<float*>(w);
   w += align_up(4 * fnc);
   __half* om = reinterpret_cast<__half*>(w);
+  uint32_t* status = pl::call_status_word();
   pl_status r = from_cuda(pl::launch_motion_kv(motion, static_cast<const __half*>(m_kv), frames,
                                                c, kv, s));
   if (r) return r;
-  r = single_gemm(x, c, m_q, c, qm, c, frames * n, c, c, nullptr, s, /*out_f32=*/true);
+  r = single_gemm(x, c, m_q, c, qm, c, frames * n, c, c, status, s, /*out_f32=*/true);
   if (r) return r;
   r = from_cuda(pl::launch_motion_attn(qm, c, kv, frames, n, c, heads, om, c, s));
   if (r) return r;
-  return single_gemm(om, c, m_o, c, out, c, frames * n, c, c, nullptr, s);
+  return single_gemm(om, c, m_o, c, out, c, frames * n, c, c, status, s);
 }
 
 pl_status pl_motion_bank_check(float* bank, int32_t* count, int32_t* appends, int capacity,
@@ -589,8 +667,10 @@ pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_
   ctx->ws_bytes = workspace_bytes;
   layout(*cfg, ctx);
   pl::ddim_coefficients(&ctx->coef);
-  // kernel attributes and the SM count are set up here, outside any stream capture
+  // kernel attributes, the SM count and the call status word are set up here,
+  // outside any stream capture
   num_sms();
+  pl::call_status_word();
   if (pl::gemm_init() || pl::attn_init()) {
     delete ctx;
     return PL_ECUDA;
@@ -881,6 +961,19 @@ pl_status pl_get_device_status(pl_ctx* ctx, void* stream) {
       return PL_ECUDA;
     w |= wz;
   }
+  if (w & pl::DEV_TIMEOUT) return PL_ETIMEOUT;
+  if (w) return PL_EDEVICE;
+  return PL_OK;
+}
+
+pl_status pl_get_call_status(void* stream) {
+  uint32_t* word = pl::call_status_word();
+  if (!word) return PL_ECUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PL_ECUDA;
+  uint32_t w = 0;
+  if (cudaMemcpy(&w, word, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return PL_ECUDA;
+  const uint32_t zero = 0;
+  if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return PL_ECUDA;
   if (w & pl::DEV_TIMEOUT) return PL_ETIMEOUT;
   if (w) return PL_EDEVICE;
   return PL_OK;

@@ -25,7 +25,13 @@
  *  - The return value reports host-side validation and launch errors only.
  *    Kernels that detect a problem on the device (a bounded wait that ran
  *    out, an argument outside the contract) set bits of a device status word
- *    instead of trapping; read it with pl_get_device_status().
+ *    instead of trapping. Calls on a context (pl_ctx, pl_sink, pl_lpm) use the
+ *    context's word: pl_get_device_status() / the state getters read it.
+ *    Calls without a context (pl_gemm_f16, pl_segment_attention,
+ *    pl_pr_sink_attention, pl_ref_attention, pl_ref_attention_noalloc,
+ *    pl_motion_xattn, pl_rope_attention) share one word per device:
+ *    pl_get_call_status() reads and clears it. After such a report the output
+ *    of the call that raised it is unspecified.
  *  - Nothing aborts, exits or traps. A context is not thread-safe.
  */
 #ifndef PL_H_
@@ -153,7 +159,10 @@ pl_status pl_ref_attention(const void* hidden, const void* w_qkv, const void* w_
  * - The call allocates nothing. Its first call on a device looks up the
  *   array's device address (cudaGetSymbolAddress) and caches it, so make that
  *   first call outside any stream capture. Every device that has made a call
- *   keeps the array until the process exits.
+ *   keeps the array until the process exits. The cached address is not looked
+ *   up again: no cudaDeviceReset may come between calls on a device.
+ * - Device-side problems go to the context-free status word
+ *   (pl_get_call_status), like those of pl_ref_attention.
  * - All calls share one array per device and it keeps the last call's
  *   contents; nothing in it has to start at zero. Calls whose execution can
  *   overlap on the GPU (other streams, other threads) race on the array:
@@ -529,6 +538,37 @@ pl_status pl_get_session_motion_bank(pl_ctx* ctx, int session, float* host_out, 
 /* Synchronise `stream` and map the device status words of all sessions to a
  * status: PL_OK, PL_ETIMEOUT or PL_EDEVICE. Clears the words. */
 pl_status pl_get_device_status(pl_ctx* ctx, void* stream);
+
+/* Synchronise `stream`, then read and clear the current device's status word
+ * of context-free calls (see the conventions above): PL_OK, PL_ETIMEOUT (a
+ * bounded wait gave up) or PL_EDEVICE (a kernel refused its arguments). The
+ * word is shared by every context-free call on the device, from any stream
+ * or thread, so a report covers all of them since the last read. The first
+ * context-free call on a device (or pl_ctx_create) looks the word's address
+ * up; make it outside stream capture. */
+pl_status pl_get_call_status(void* stream);
+
+/* ------------------------------------------------------------------ *
+ * Test hooks (no counterpart in the pages): planted device-side failures
+ * that exercise the error paths without faulting or hanging the GPU.
+ * ------------------------------------------------------------------ */
+
+#define PL_TEST_NO_KV 1    /* the producer loads Q but no K/V tile */
+#define PL_TEST_BAD_BOX 2  /* the kernel is told a K/V box that is not its tile */
+
+/* pl_segment_attention with a planted failure. PL_TEST_NO_KV: no K/V copy is
+ * started, so the MMA issuers' bounded waits run out after wait_us
+ * microseconds (1..2000000); the kernel raises its abort flag, every role
+ * leaves its loop, TMEM is freed and the call status becomes PL_ETIMEOUT.
+ * PL_TEST_BAD_BOX: the box count the kernel checks is off by 16 rows (the
+ * tensor maps themselves are right), so every CTA returns before any copy
+ * and the call status becomes PL_EDEVICE. `out` is not written in either
+ * mode. Arguments as for pl_segment_attention. */
+pl_status pl_test_segment_attention_fault(const void* q, int64_t ldq, int64_t q_frame_stride,
+                                         const pl_kv_segment* segs, int n_segs, int frames,
+                                         int n_q, int heads, int head_dim, void* out,
+                                         int64_t ldo, int64_t out_frame_stride, int mode,
+                                         uint32_t wait_us, void* stream);
 
 /* Device pointer of the piles' latents, fp32 [S][4 slots][4][4][H][W]
  * (read-only view for tests; slot s holds the window at timestep slot_t[s]). */

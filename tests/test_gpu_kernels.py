@@ -68,6 +68,24 @@ def test_segment_attention_peaky_scores(P):
     assert mx <= 3e-2 and rel < 1e-2, (mx, mean, rel)
 
 
+@pytest.mark.parametrize("hd", [40, 64])
+@pytest.mark.parametrize("L", [1, 50, 80, 81, 161])
+def test_segment_attention_few_key_tiles(P, hd, L):
+    # one or two key tiles in all (a single key, a partial tile, exactly one
+    # or two tiles, one key past a tile): the first tile's maximum starts the
+    # running maximum and the last, mostly masked tile ends it
+    F, Nq, heads = 2, 300, 2
+    Cc = heads * hd
+    q = S.normal(44, f"q{hd}{L}", (F, Nq, Cc), 1.0, np.float16)
+    k = S.normal(44, f"k{hd}{L}", (F, L, Cc), 1.0, np.float16)
+    v = S.normal(44, f"v{hd}{L}", (F, L, Cc), 1.0, np.float16)
+    got = host(P.segment_attention(dev(q), [(dev(k), dev(v))], heads, hd)).astype(np.float64)
+    for f in range(F):
+        want = O.segment_attention(q[f], [k[f]], [v[f]], heads)
+        mx, mean, rel = attn_errors(got[f], want)
+        assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (f, mx, mean, rel)
+
+
 @pytest.mark.parametrize("hd", [40, 80, 128, 160])
 @pytest.mark.parametrize("shape", ["ramp", "spikes"])
 def test_segment_attention_growing_max(P, hd, shape):

@@ -365,6 +365,28 @@ def test_motion_pe_structure():
     assert np.max(np.abs(pe[:, 1] - np.cos(p))) < 1e-15
 
 
+def test_motion_pe_hand_values_at_later_pairs():
+    # literal values of later pairs (golden file): an exponent i/d instead of
+    # 2i/d, a swapped sin/cos or a shifted pair index fails here
+    path = os.path.join(os.path.dirname(__file__), "golden", "motion_pe_values.txt")
+    pe = O.motion_pe()
+    rows = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    assert len(rows) == 8
+    for p, c, v in rows:
+        assert abs(pe[int(p), int(c)] - float(v)) < 1e-14, (p, c)
+
+
+def test_motion_pe_frequency_drops_a_decade_every_two_pairs():
+    # pair i + 2 turns ten times slower than pair i (10000^(-2(i+2)/16) =
+    # 10000^(-2i/16) / 10), so position 10p on pair i + 2 repeats position p
+    # on pair i; with any other exponent the decade lands elsewhere
+    pe = O.motion_pe()
+    for p in (1, 2, 3):
+        for i in range(6):
+            assert abs(pe[10 * p, 2 * (i + 2)] - pe[p, 2 * i]) < 1e-12, (p, i)
+            assert abs(pe[10 * p, 2 * (i + 2) + 1] - pe[p, 2 * i + 1]) < 1e-12, (p, i)
+
+
 def test_motion_tokens_reshape_is_row_major():
     e = np.arange(512, dtype=np.float64)
     tok = O.motion_tokens(e) - O.motion_pe()
@@ -530,6 +552,20 @@ def test_dot_image_disc_and_painter_order():
     # overlapping dots: the later one wins where both cover
     img = O.dot_image(np.array([[3.5, 2.5], [4.5, 2.5]]), col, 1.0, 6, 8)
     assert img[1, 2, 4] == 1 and img[0, 2, 4] == 0 and img[0, 2, 2] == 1
+
+
+def test_dot_centres_corners_and_centre_on_a_wide_image():
+    # orthographic map of [-1, 1] x [-1, 1] onto [0, W] x [0, H] with H != W,
+    # so a swapped axis, a missing half-width or a half-pixel shift fails
+    H, W = 48, 80
+    kps = np.array([[-1.0, -1.0, 0.3], [1.0, 1.0, -0.2], [0.0, 0.0, 5.0], [1.0, -1.0, 0.0],
+                    [-1.0, 1.0, 0.0], [0.5, -0.5, 0.0], [-0.25, 0.75, 0.0], [9.0, 9.0, 9.0]])
+    got = O.dot_centres(kps, [0, 1, 2, 3, 4, 5, 6], H, W)
+    want = np.array([[0.0, 0.0], [80.0, 48.0], [40.0, 24.0], [80.0, 0.0], [0.0, 48.0],
+                     [60.0, 12.0], [30.0, 42.0]])
+    assert np.array_equal(got, want)
+    # the selection picks rows in the order given
+    assert np.array_equal(O.dot_centres(kps, [2, 0], H, W), want[[2, 0]])
 
 
 def test_prefill_keypoints_ramp():
