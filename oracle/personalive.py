@@ -187,24 +187,33 @@ def motion_tokens(e: np.ndarray) -> np.ndarray:
     return e + motion_pe()
 
 
-def motion_xattn_frame(x: np.ndarray, tokens: np.ndarray, w: dict, heads: int) -> np.ndarray:
+def motion_xattn_frame(x: np.ndarray, tokens: np.ndarray, w: dict, heads: int,
+                       block: int = 1) -> np.ndarray:
     """Cross-attention of one frame's tokens to its 32 motion tokens.
 
     cross_attention_dim 16, 8 heads: Q = x Mq ([C,C]), K = m Mk, V = m Mv
-    ([16, C]), out = softmax(Q K^T / sqrt(hd)) V Mo.
+    ([16, C]), out = softmax(Q K^T / sqrt(hd)) V Mo. Block 1 uses the
+    weights mq, mk, mv, mo; block b > 1 uses mq<b>, mk<b>, mv<b>, mo<b>.
     """
+    sfx = "" if block == 1 else str(block)
     x = np.asarray(x, np.float64)
     m = np.asarray(tokens, np.float64)
-    q = x @ np.asarray(w["mq"], np.float64)
-    k = m @ np.asarray(w["mk"], np.float64)
-    v = m @ np.asarray(w["mv"], np.float64)
-    return mha(q, k, v, heads) @ np.asarray(w["mo"], np.float64)
+    q = x @ np.asarray(w["mq" + sfx], np.float64)
+    k = m @ np.asarray(w["mk" + sfx], np.float64)
+    v = m @ np.asarray(w["mv" + sfx], np.float64)
+    return mha(q, k, v, heads) @ np.asarray(w["mo" + sfx], np.float64)
 
 
-def layer_forward_frame(h, w, bank, tokens, heads, rows=None):
-    """One reference-attention layer followed by its motion cross-attention."""
+def layer_forward_frame(h, w, bank, tokens, heads, rows=None, motion_blocks=1):
+    """One reference-attention layer followed by its motion cross-attention
+    block(s). [PL] "三条条件通路" lists the motion module's attention blocks as
+    [Spatial_Cross, Spatial_Cross]; with motion_blocks = 2 the second block
+    (own weights, same 32 tokens) takes the first block's output as its
+    queries, the way each sub-layer consumes the previous one's result."""
     a = ref_attention_frame(h, w, bank, heads, rows=rows)
-    return motion_xattn_frame(a, tokens, w, heads)
+    for b in range(1, motion_blocks + 1):
+        a = motion_xattn_frame(a, tokens, w, heads, block=b)
+    return a
 
 
 # ---------------------------------------------------------------------------

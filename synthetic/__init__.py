@@ -112,6 +112,21 @@ def layer_weights(seed: int, layer: str, C: int, dtype=np.float16):
     }
 
 
+def motion_block_weights(seed: int, layer: str, C: int, block: int, dtype=np.float16):
+    """Weights of motion cross-attention block `block` (2, ...) of a layer, as
+    layer_weights draws block 1's: mq, mo [C, C] N(0, 1/C); mk, mv [16, C]
+    N(0, 1/16). Keys carry the block number (mq2, mk2, ...)."""
+    s_c = 1.0 / np.sqrt(C)
+    s_m = 1.0 / np.sqrt(MOTION_TOKEN_DIM)
+    b = int(block)
+    return {
+        f"mq{b}": normal(seed, f"{layer}/mq{b}", (C, C), s_c, dtype),
+        f"mk{b}": normal(seed, f"{layer}/mk{b}", (MOTION_TOKEN_DIM, C), s_m, dtype),
+        f"mv{b}": normal(seed, f"{layer}/mv{b}", (MOTION_TOKEN_DIM, C), s_m, dtype),
+        f"mo{b}": normal(seed, f"{layer}/mo{b}", (C, C), s_c, dtype),
+    }
+
+
 def layer_hidden(seed: int, layer: str, round_idx: int, F: int, N: int, C: int,
                  scale: float = 1.0, dtype=np.float16):
     """Per-round `norm_hidden_states` stand-in, N(0, scale^2), [F, N, C]."""

@@ -403,6 +403,47 @@ def test_motion_xattn_identical_tokens():
     assert np.max(np.abs(got - want[None])) < 1e-12
 
 
+def test_two_motion_blocks_with_identical_tokens():
+    # with 32 identical tokens each block returns the constant row (m Mv) Mo
+    # whatever its queries, so the layer's output is block 2's constant row
+    # (own weights, not block 1's) and block 1's queries do not matter
+    C = 32
+    w = S.layer_weights(24, "mx", C, np.float64)
+    w.update(S.motion_block_weights(24, "mx", C, 2, np.float64))
+    m = np.tile(S.normal(24, "m", (16,)), (32, 1))
+    h = S.normal(24, "h", (6, C))
+    bank = [S.normal(24, "b", (6, C))]
+    got = O.layer_forward_frame(h, w, bank, m, 8, motion_blocks=2)
+    want2 = (m[0] @ w["mv2"]) @ w["mo2"]
+    want1 = (m[0] @ w["mv"]) @ w["mo"]
+    assert np.max(np.abs(got - want2[None])) < 1e-12
+    assert np.max(np.abs(want2 - want1)) > 1e-3          # the blocks' weights differ
+
+
+def test_second_motion_block_takes_the_first_blocks_output():
+    # identical tokens in block 1 make every row of its output the same, so
+    # block 2 (varied tokens) must see identical query rows and return
+    # identical rows; fed the reference-attention output instead (rows
+    # differ) it would not
+    C = 32
+    w = S.layer_weights(25, "mx", C, np.float64)
+    w.update(S.motion_block_weights(25, "mx", C, 2, np.float64))
+    h = S.normal(25, "h", (6, C))
+    bank = [S.normal(25, "b", (6, C))]
+    a = O.ref_attention_frame(h, w, bank, 8)
+    m1 = np.tile(S.normal(25, "m1", (16,)), (32, 1))
+    m_var = S.normal(25, "mvar", (32, 16))
+    y1 = O.motion_xattn_frame(a, m1, w, 8)
+    assert np.max(np.abs(y1 - y1[0][None])) < 1e-12
+    y2 = O.motion_xattn_frame(y1, m_var, w, 8, block=2)
+    assert np.max(np.abs(y2 - y2[0][None])) < 1e-12
+    assert np.max(np.abs(O.motion_xattn_frame(a, m_var, w, 8, block=2)[1:] -
+                         O.motion_xattn_frame(a, m_var, w, 8, block=2)[0])) > 1e-3
+    # motion_blocks = 1 is the single block of the round
+    one = O.layer_forward_frame(h, w, bank, m_var, 8)
+    assert np.array_equal(one, O.motion_xattn_frame(a, m_var, w, 8))
+
+
 def test_motion_xattn_brute_force():
     C = 16
     w = S.layer_weights(24, "mx", C, np.float64)
