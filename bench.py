@@ -533,8 +533,9 @@ def secondary_measurements(torch, P, stream, hbm_peak):
     """The other workloads' kernels, timed live (CUDA events on their stream):
     the PR-Sink block (4096 tokens x 40 heads x 128, KV own + sink + retrieved
     of 64 + 3 rolling), the pile DDIM step on a scaled latent grid (1024 x 1024:
-    ring + epsilon 512 MB, past L2), and the nearest-vector search over a 1 GB
-    store. Inputs are seeded torch tensors (timing only)."""
+    ring + epsilon 512 MB, past L2), the nearest-vector search over a 1 GB
+    store and the motion-bank check of 4 embeddings over a 512 MB bank.
+    Inputs are seeded torch tensors (timing only)."""
     g = torch.Generator(device="cuda").manual_seed(SEED)
     out = {}
     # PR-Sink
@@ -585,6 +586,23 @@ def secondary_measurements(torch, P, stream, hbm_peak):
     out["nearest_2M_x128"] = {"ms": t * 1e3, "gbs": byts / t / 1e9,
                               "frac_hbm": byts / t / 1e9 / hbm_peak}
     del store
+    # motion-bank check at scale: 4 round embeddings checked in order against a
+    # full bank of 262144 x 512 (512 MB, past L2; full, so no append changes
+    # the work between calls)
+    count, dim = 1 << 18, 512
+    bank = 2.0 * torch.randn((count, dim), device="cuda", generator=g)
+    qs = 2.0 * torch.randn((4, dim), device="cuda", generator=g)
+    cnt = torch.full((1,), count, dtype=torch.int32, device="cuda")
+    app = torch.zeros(1, dtype=torch.int32, device="cuda")
+    need = P.sz()
+    P.check(P.lib.pl_motion_bank_check_workspace_bytes(count, dim, 4, P.C.byref(need)), "ws")
+    ws = torch.empty(need.value, dtype=torch.uint8, device="cuda")
+    t = _event_time(torch, lambda: P.motion_bank_check(bank, cnt, app, qs, 17.0, 3, workspace=ws,
+                                                       stream=stream), 10, stream)
+    byts = 4.0 * (count + 4) * dim
+    out["bank_check_256k_x512_q4"] = {"ms": t * 1e3, "gbs": byts / t / 1e9,
+                                      "frac_hbm": byts / t / 1e9 / hbm_peak}
+    del bank
     torch.cuda.synchronize()
     return out
 

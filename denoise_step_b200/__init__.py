@@ -41,7 +41,7 @@ class Config(C.Structure):
                 ("n_layers", C.c_int32), ("layer_tokens", C.c_int32 * MAX_LAYERS),
                 ("layer_channels", C.c_int32 * MAX_LAYERS), ("heads", C.c_int32),
                 ("drift_threshold", C.c_float), ("append_cap", C.c_int32),
-                ("sessions", C.c_int32)]
+                ("sessions", C.c_int32), ("motion_blocks", C.c_int32)]
 
 
 class SinkState(C.Structure):
@@ -62,7 +62,8 @@ class LpmState(C.Structure):
 
 
 class LayerWeights(C.Structure):
-    _fields_ = [("w_qkv", vp), ("w_o", vp), ("m_q", vp), ("m_kv", vp), ("m_o", vp)]
+    _fields_ = [("w_qkv", vp), ("w_o", vp), ("m_q", vp), ("m_kv", vp), ("m_o", vp),
+                ("m2_q", vp), ("m2_kv", vp), ("m2_o", vp)]
 
 
 class State(C.Structure):
@@ -93,7 +94,9 @@ _SIGS = {
     "pl_ref_attention_noalloc": (i32, [vp, vp, vp, C.POINTER(vp), i32, i32, i32, i32, i32, vp, vp]),
     "pl_motion_xattn_workspace_bytes": (i32, [i32, i32, i32, C.POINTER(sz)]),
     "pl_motion_xattn": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, sz, vp]),
-    "pl_motion_bank_check": (i32, [vp, vp, vp, i32, i32, vp, i32, f32, i32, vp, vp, vp, vp]),
+    "pl_motion_bank_check_workspace_bytes": (i32, [i32, i32, i32, C.POINTER(sz)]),
+    "pl_motion_bank_check": (i32, [vp, vp, vp, i32, i32, vp, i32, f32, i32, vp, vp, vp, vp, sz,
+                                   vp]),
     "pl_nearest_workspace_bytes": (i32, [i64, C.POINTER(sz)]),
     "pl_nearest": (i32, [vp, i64, i32, vp, vp, vp, vp, sz, vp]),
     "pl_workspace_bytes": (i32, [C.POINTER(Config), C.POINTER(sz)]),
@@ -104,7 +107,8 @@ _SIGS = {
     "pl_ring_push": (i32, [vp, vp, vp, vp]),
     "pl_pyramid_ddim_step": (i32, [vp, vp, vp, vp]),
     "pl_ctx_bank_check": (i32, [vp, vp, i32, vp, vp, vp, vp]),
-    "pl_stream_round": (i32, [vp, vp, vp, C.POINTER(vp), vp, vp, vp, C.POINTER(vp), vp]),
+    "pl_stream_round": (i32, [vp, vp, vp, C.POINTER(vp), vp, vp, vp, C.POINTER(vp),
+                              C.POINTER(vp), vp]),
     "pl_host_staging_bytes": (i32, [C.POINTER(Config), C.POINTER(sz)]),
     "pl_stream_round_host": (i32, [vp, vp, sz, vp, vp, C.POINTER(vp), vp, vp, vp]),
     "pl_get_state": (i32, [vp, C.POINTER(State), vp]),
@@ -300,13 +304,22 @@ def motion_xattn(x, motion, m_q, m_kv, m_o, heads, out=None, workspace=None, str
 
 
 def motion_bank_check(bank, count, appends, queries, threshold, cap, argmin=None, min_d2=None,
-                      appended=None, stream=None):
-    """In-order bank check; bank [capacity, dim] fp32, count/appends int32 [1] (device state)."""
+                      appended=None, workspace=None, stream=None):
+    """In-order bank check; bank [capacity, dim] fp32, count/appends int32 [1] (device state).
+    Banks past 32 entries (or more than 32 queries) need a device workspace; it is
+    allocated here when not given."""
+    import torch
     cap_, dim = bank.shape
     nq = queries.shape[0]
+    need = sz()
+    check(lib.pl_motion_bank_check_workspace_bytes(cap_, dim, nq, C.byref(need)), "workspace")
+    if workspace is None and need.value > 0:
+        workspace = torch.empty(need.value, dtype=torch.uint8, device=bank.device)
+    wb = workspace.numel() if workspace is not None else 0
     check(lib.pl_motion_bank_check(_ptr(bank), _ptr(count), _ptr(appends), cap_, dim,
                                    _ptr(queries), nq, float(threshold), int(cap), _ptr(argmin),
-                                   _ptr(min_d2), _ptr(appended), _stream(stream)),
+                                   _ptr(min_d2), _ptr(appended), _ptr(workspace), wb,
+                                   _stream(stream)),
           "pl_motion_bank_check")
 
 
@@ -331,8 +344,9 @@ def nearest(store, query, argmin=None, min_d2=None, workspace=None, stream=None)
 # --------------------------------------------------------------------------- stream context
 
 def make_config(latent_hw=(64, 64), layers=(), heads=8, threshold=17.0, append_cap=3, latent_c=4,
-                sessions=1):
-    """layers: sequence of (tokens N, channels C); sessions: streams served together."""
+                sessions=1, motion_blocks=1):
+    """layers: sequence of (tokens N, channels C); sessions: streams served together;
+    motion_blocks: motion cross-attention blocks per layer (1 or 2)."""
     cfg = Config()
     cfg.latent_c, (cfg.latent_h, cfg.latent_w) = latent_c, latent_hw
     cfg.n_layers = len(layers)
@@ -343,6 +357,7 @@ def make_config(latent_hw=(64, 64), layers=(), heads=8, threshold=17.0, append_c
     cfg.drift_threshold = threshold
     cfg.append_cap = append_cap
     cfg.sessions = sessions
+    cfg.motion_blocks = motion_blocks
     return cfg
 
 
@@ -378,12 +393,14 @@ class Stream:
 
     def bank_init(self, weights, ref_feats, anchor_feats, ref_motion, drive0_motion, ref_latent,
                   prefill_eps, stream=None):
-        """weights: list of dicts with w_qkv, w_o, m_q, m_kv, m_o (device fp16)."""
+        """weights: list of dicts with w_qkv, w_o, m_q, m_kv, m_o (device fp16), and
+        m2_q, m2_kv, m2_o for a second motion block."""
         L = self.cfg.n_layers
         wa = (LayerWeights * max(L, 1))()
         for i, w in enumerate(weights[:L]):
             wa[i] = LayerWeights(_ptr(w["w_qkv"]), _ptr(w["w_o"]), _ptr(w["m_q"]),
-                                 _ptr(w["m_kv"]), _ptr(w["m_o"]))
+                                 _ptr(w["m_kv"]), _ptr(w["m_o"]), _ptr(w.get("m2_q")),
+                                 _ptr(w.get("m2_kv")), _ptr(w.get("m2_o")))
         rf = _ptr_array(ref_feats) if L else None
         af = _ptr_array(anchor_feats) if anchor_feats else None
         self._keep = [weights, ref_feats, anchor_feats, ref_motion, drive0_motion, ref_latent,
@@ -406,12 +423,14 @@ class Stream:
               "pl_ctx_bank_check")
 
     def round(self, new_noise, new_motion, hidden, eps, out_frames, appended=None,
-              layer_out=None, stream=None):
+              layer_out=None, stream=None, attn_out=None):
+        """attn_out: optional per-layer buffers for the reference-attention sub-layer output."""
         L = self.cfg.n_layers
         hp = _ptr_array(hidden) if L else None
         lo = _ptr_array(layer_out) if layer_out is not None else None
+        ao = _ptr_array(attn_out) if attn_out is not None else None
         check(lib.pl_stream_round(self.handle, _ptr(new_noise), _ptr(new_motion), hp, _ptr(eps),
-                                  _ptr(out_frames), _ptr(appended), lo, _stream(stream)),
+                                  _ptr(out_frames), _ptr(appended), lo, ao, _stream(stream)),
               "pl_stream_round")
 
     def round_host(self, h_noise, h_motion, h_hidden, h_eps, h_out_frames, stream=None):

@@ -197,15 +197,87 @@ __global__ void ring_commit_kernel(DevState* st) {
 }
 
 // ------------------------------------------------------------------ bank check
+// In-order bank check ([PL] 抗身份漂移的补丁): query k sees the stored entries
+// and the queries appended before it in the same call. An appended entry is
+// the query itself, bit for bit, so every distance the check can need is one
+// of two kinds, both fixed before any decision: query k to a stored entry j,
+// and query k to an earlier query i. They are computed in one parallel pass
+// (fp64 from the fp32 values, one warp per pair or per entry); the decisions
+// then run in order over that table: nearest stored entry (lowest index on
+// ties), then the earlier appended queries in their append order (their bank
+// indices follow the stored ones); append when d^2 > thr^2, the cap allows
+// it and the bank has room.
 constexpr int kBankThreads = 256;
+constexpr int kBankSmall = 32;     // capacity and queries of the one-CTA path
 
+// squared distance of two fp32 vectors in fp64, summed over the warp (every
+// lane gets the total)
+__device__ __forceinline__ double dist2_warp(const float* a, const float* b, int dim, int lane) {
+  double acc = 0.0;
+  const bool vec = (dim & 3) == 0 &&
+                   ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 15) == 0;
+  if (vec) {
+    for (int d = 4 * lane; d < dim; d += 128) {
+      const float4 x = *reinterpret_cast<const float4*>(a + d);
+      const float4 y = *reinterpret_cast<const float4*>(b + d);
+      const double d0 = static_cast<double>(x.x) - y.x, d1 = static_cast<double>(x.y) - y.y;
+      const double d2 = static_cast<double>(x.z) - y.z, d3 = static_cast<double>(x.w) - y.w;
+      acc = fma(d3, d3, fma(d2, d2, fma(d1, d1, fma(d0, d0, acc))));
+    }
+  } else {
+    for (int d = lane; d < dim; d += 32) {
+      const double df = static_cast<double>(a[d]) - b[d];
+      acc = fma(df, df, acc);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc;
+}
+
+// Decisions of one call, in query order, from the existing-entry minima (per
+// query: d2 and index, index -1 when the bank is empty) and the query-query
+// table dq[k * ldq + i] (i < k). Run by one thread. Returns the appends made;
+// list[a] = query appended a-th.
+__device__ int bank_decide(const double* e_d2, const int* e_idx, const double* dq, int ldq,
+                           int nq, int cnt0, int app0, int capacity, double thr2, int cap,
+                           int32_t* argmin, double* min_d2, uint8_t* appended, int* list,
+                           DevState* st) {
+  int cnt = cnt0, app = app0, n_app = 0;
+  for (int k = 0; k < nq; ++k) {
+    double best = e_d2[k];
+    int bi = e_idx[k];
+    for (int a = 0; a < n_app; ++a) {
+      const double d = dq[k * ldq + list[a]];
+      if (d < best) {   // appended entries come after the stored ones
+        best = d;
+        bi = cnt0 + a;
+      }
+    }
+    if (argmin) argmin[k] = bi;
+    if (min_d2) min_d2[k] = best;
+    const bool doit = cnt > 0 && best > thr2 && app < cap && cnt < capacity;
+    if (appended) appended[k] = doit ? 1 : 0;
+    if (doit) {
+      list[n_app++] = k;
+      ++cnt;
+      ++app;
+      if (st && app < 4) st->anchor_fire[app] = 1;
+    }
+  }
+  return n_app;
+}
+
+// One CTA per session (the round's check; capacity and queries <= kBankSmall).
 __global__ void __launch_bounds__(kBankThreads) bank_check_kernel(
     float* bank, int32_t* count_p, int32_t* appends_p, int capacity, int dim,
     const float* __restrict__ queries, int nq, double thr2, int cap, int32_t* argmin,
-    double* min_d2, uint8_t* appended, DevState* st, int count_val) {
-  __shared__ double w_best[kBankThreads / 32];
-  __shared__ int w_idx[kBankThreads / 32];
-  __shared__ int s_cnt, s_app, s_do_append;
+    double* min_d2, uint8_t* appended, DevState* st) {
+  __shared__ double s_de[kBankSmall * kBankSmall];   // [k][j]: query k, stored entry j
+  __shared__ double s_dq[kBankSmall * kBankSmall];   // [k][i]: query k, earlier query i
+  __shared__ double s_bd[kBankSmall];
+  __shared__ int s_bi[kBankSmall], s_list[kBankSmall];
+  __shared__ int s_cnt0, s_app0, s_napp;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int nwarps = kBankThreads / 32;
   if (st) {
@@ -221,69 +293,316 @@ __global__ void __launch_bounds__(kBankThreads) bank_check_kernel(
     if (appended) appended += z * nq;
   }
   if (threadIdx.x == 0) {
-    s_cnt = count_p ? *count_p : count_val;
-    s_app = appends_p ? *appends_p : 0;
-    if (st) {
+    int c = *count_p;
+    s_cnt0 = c < 0 ? 0 : (c > capacity ? capacity : c);
+    s_app0 = *appends_p;
+    if (st)
       for (int a = 0; a < 4; ++a) st->anchor_fire[a] = 0;
+  }
+  __syncthreads();
+  const int cnt0 = s_cnt0;
+  const int n_e = nq * cnt0, n_all = n_e + nq * nq;
+  for (int p = warp; p < n_all; p += nwarps) {
+    int k, j;
+    const float* b;
+    if (p < n_e) {
+      k = p / cnt0;
+      j = p - k * cnt0;
+      b = bank + static_cast<int64_t>(j) * dim;
+    } else {
+      k = (p - n_e) / nq;
+      j = (p - n_e) - k * nq;
+      if (j >= k) continue;   // warp-uniform
+      b = queries + static_cast<int64_t>(j) * dim;
+    }
+    const double d = dist2_warp(queries + static_cast<int64_t>(k) * dim, b, dim, lane);
+    if (lane == 0) (p < n_e ? s_de : s_dq)[k * kBankSmall + j] = d;
+  }
+  __syncthreads();
+  if (threadIdx.x < nq) {
+    // nearest stored entry of query threadIdx.x (ascending j, strict <)
+    const int k = threadIdx.x;
+    double b = INFINITY;
+    int bi = -1;
+    for (int j = 0; j < cnt0; ++j)
+      if (s_de[k * kBankSmall + j] < b) {
+        b = s_de[k * kBankSmall + j];
+        bi = j;
+      }
+    s_bd[k] = b;
+    s_bi[k] = bi;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int n_app = bank_decide(s_bd, s_bi, s_dq, kBankSmall, nq, cnt0, s_app0, capacity, thr2,
+                                  cap, argmin, min_d2, appended, s_list, st);
+    s_napp = n_app;
+    *count_p = cnt0 + n_app;
+    *appends_p = s_app0 + n_app;
+  }
+  __syncthreads();
+  for (int a = 0; a < s_napp; ++a) {
+    const float* src = queries + static_cast<int64_t>(s_list[a]) * dim;
+    float* dst = bank + static_cast<int64_t>(cnt0 + a) * dim;
+    for (int d = threadIdx.x; d < dim; d += kBankThreads) dst[d] = src[d];
+  }
+}
+
+// Large banks, pass 1: each CTA takes a slice of the stored entries and keeps,
+// per query, its nearest entry (lowest index on ties). Every entry is read
+// once for all queries; the queries sit in shared memory as fp64. Four lanes
+// share an entry: each lane walks its quarter of the row in 16-byte chunks,
+// so a warp load covers 8 rows x 64 contiguous bytes (whole sectors), the
+// four lanes of an entry read different query values and the eight entries
+// the same ones (broadcast, no bank conflict), and an entry's sum needs two
+// shuffle steps. Each lane takes kBankE entries at once (slot + 8 e), so a
+// query value read from shared memory serves kBankE entries: with one it
+// was the shared-memory reads that bound the pass (L1 pipe 82%). Measured
+// alternatives at 262144 x 512 with 4 queries: a warp per entry (five-step
+// reduction per entry and query, 124 registers) and a thread per entry (32
+// rows per warp load, L1-bound at 93%) both ran at ~2.2 TB/s.
+constexpr int kBankGroup = 4;
+constexpr int kBankLanes = 4;              // lanes per entry
+constexpr int kBankE = 4;                  // entries per lane at once (2 measured slower)
+constexpr int kBankMaxQueries = 64;
+
+__global__ void __launch_bounds__(kBankThreads) bank_partial_kernel(
+    const float* __restrict__ bank, const int32_t* count_p, int64_t capacity, int dim,
+    const float* __restrict__ queries, int nq, double* part_d2, int64_t* part_idx) {
+  extern __shared__ double sq[];                    // [nq][dim]
+  __shared__ double w_best[kBankThreads / 32][kBankMaxQueries];
+  __shared__ int64_t w_idx[kBankThreads / 32][kBankMaxQueries];
+  constexpr int kSlots = 32 / kBankLanes;
+  constexpr int kPerWarp = kSlots * kBankE;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane % kBankLanes, slot = lane / kBankLanes;
+  for (int i = threadIdx.x; i < nq * dim; i += kBankThreads) sq[i] = static_cast<double>(queries[i]);
+  __syncthreads();
+  int64_t cnt = *count_p;
+  cnt = cnt < 0 ? 0 : (cnt > capacity ? capacity : cnt);
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * (kBankThreads / 32) + warp;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (kBankThreads / 32);
+  const bool vec = (dim & 3) == 0 && (reinterpret_cast<uintptr_t>(bank) & 15) == 0;
+  for (int g0 = 0; g0 < nq; g0 += kBankGroup) {
+    const int gn = nq - g0 < kBankGroup ? nq - g0 : kBankGroup;
+    const double* q0 = sq + static_cast<int64_t>(g0) * dim;
+    double best[kBankGroup];
+    int64_t bidx[kBankGroup];
+#pragma unroll
+    for (int g = 0; g < kBankGroup; ++g) {
+      best[g] = INFINITY;
+      bidx[g] = -1;
+    }
+    for (int64_t j0 = gw * kPerWarp; j0 < cnt; j0 += nw * kPerWarp) {
+      // a lane's entries: j0 + slot + kSlots * u, increasing
+      double acc[kBankE][kBankGroup];
+#pragma unroll
+      for (int u = 0; u < kBankE; ++u)
+#pragma unroll
+        for (int g = 0; g < kBankGroup; ++g) acc[u][g] = 0.0;
+      const float* e[kBankE];
+      bool ok[kBankE];
+#pragma unroll
+      for (int u = 0; u < kBankE; ++u) {
+        const int64_t j = j0 + slot + kSlots * u;
+        ok[u] = j < cnt;
+        e[u] = bank + (ok[u] ? j : 0) * dim;   // rows past the end read row 0, unused
+      }
+      if (vec) {
+#pragma unroll 2
+        for (int d = 4 * sub; d < dim; d += 4 * kBankLanes) {
+          double x[kBankE][4];
+#pragma unroll
+          for (int u = 0; u < kBankE; ++u) {
+            const float4 t = __ldg(reinterpret_cast<const float4*>(e[u] + d));
+            x[u][0] = t.x;
+            x[u][1] = t.y;
+            x[u][2] = t.z;
+            x[u][3] = t.w;
+          }
+#pragma unroll
+          for (int g = 0; g < kBankGroup; ++g) {
+            if (g < gn) {
+              const double2 qa = *reinterpret_cast<const double2*>(q0 + g * dim + d);
+              const double2 qb = *reinterpret_cast<const double2*>(q0 + g * dim + d + 2);
+#pragma unroll
+              for (int u = 0; u < kBankE; ++u) {
+                const double d0 = qa.x - x[u][0], d1 = qa.y - x[u][1];
+                const double d2 = qb.x - x[u][2], d3 = qb.y - x[u][3];
+                acc[u][g] = fma(d3, d3, fma(d2, d2, fma(d1, d1, fma(d0, d0, acc[u][g]))));
+              }
+            }
+          }
+        }
+      } else {
+        for (int d = sub; d < dim; d += kBankLanes) {
+          double x[kBankE];
+#pragma unroll
+          for (int u = 0; u < kBankE; ++u) x[u] = e[u][d];
+#pragma unroll
+          for (int g = 0; g < kBankGroup; ++g)
+            if (g < gn) {
+              const double q = q0[g * dim + d];
+#pragma unroll
+              for (int u = 0; u < kBankE; ++u) {
+                const double df = q - x[u];
+                acc[u][g] = fma(df, df, acc[u][g]);
+              }
+            }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBankE; ++u) {
+#pragma unroll
+        for (int g = 0; g < kBankGroup; ++g) {
+          if (g < gn) {
+#pragma unroll
+            for (int o = 1; o < kBankLanes; o <<= 1)
+              acc[u][g] += __shfl_xor_sync(0xffffffffu, acc[u][g], o);
+            if (ok[u] && acc[u][g] < best[g]) {
+              best[g] = acc[u][g];
+              bidx[g] = j0 + slot + kSlots * u;
+            }
+          }
+        }
+      }
+    }
+    // warp minimum per query (lowest index on ties), then one entry per warp
+#pragma unroll
+    for (int g = 0; g < kBankGroup; ++g) {
+      if (g < gn) {
+        double b = best[g];
+        int64_t bi = bidx[g];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const double ob = __shfl_xor_sync(0xffffffffu, b, o);
+          const int64_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+          if (oi >= 0 && (bi < 0 || ob < b || (ob == b && oi < bi))) {
+            b = ob;
+            bi = oi;
+          }
+        }
+        if (lane == 0) {
+          w_best[warp][g0 + g] = b;
+          w_idx[warp][g0 + g] = bi;
+        }
+      }
     }
   }
   __syncthreads();
-  for (int qi = 0; qi < nq; ++qi) {
-    const float* q = queries + static_cast<int64_t>(qi) * dim;
-    const int cnt = s_cnt;
-    double best = INFINITY;
-    int bidx = 0x7fffffff;
-    for (int j = warp; j < cnt; j += nwarps) {
-      const float* b = bank + static_cast<int64_t>(j) * dim;
-      double acc = 0.0;
-      for (int d = lane; d < dim; d += 32) {
-        const double diff = static_cast<double>(q[d]) - static_cast<double>(b[d]);
-        acc = fma(diff, diff, acc);
+  for (int k = threadIdx.x; k < nq; k += kBankThreads) {
+    double b = INFINITY;
+    int64_t bi = -1;
+    for (int w = 0; w < kBankThreads / 32; ++w) {
+      const int64_t wi = w_idx[w][k];
+      if (wi >= 0 && (bi < 0 || w_best[w][k] < b || (w_best[w][k] == b && wi < bi))) {
+        b = w_best[w][k];
+        bi = wi;
       }
+    }
+    part_d2[static_cast<int64_t>(blockIdx.x) * nq + k] = b;
+    part_idx[static_cast<int64_t>(blockIdx.x) * nq + k] = bi;
+  }
+}
+
+// Large banks, pass 2 (one CTA): per query the minimum over the partial
+// minima, the query-query distances, the in-order decisions and the copies.
+__global__ void __launch_bounds__(kBankThreads) bank_resolve_kernel(
+    float* bank, int32_t* count_p, int32_t* appends_p, int capacity, int dim,
+    const float* __restrict__ queries, int nq, double thr2, int cap, const double* part_d2,
+    const int64_t* part_idx, int parts, int32_t* argmin, double* min_d2, uint8_t* appended) {
+  __shared__ double s_dq[kBankMaxQueries * kBankMaxQueries];
+  __shared__ double s_bd[kBankMaxQueries];
+  __shared__ int s_bi[kBankMaxQueries], s_list[kBankMaxQueries];
+  __shared__ int s_cnt0, s_app0, s_napp;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int nwarps = kBankThreads / 32;
+  if (threadIdx.x == 0) {
+    const int c = *count_p;
+    s_cnt0 = c < 0 ? 0 : (c > capacity ? capacity : c);
+    s_app0 = *appends_p;
+  }
+  // per query: one warp reduces the partial minima (lowest index on ties)
+  for (int k = warp; k < nq; k += nwarps) {
+    double b = INFINITY;
+    int64_t bi = -1;
+    for (int pt = lane; pt < parts; pt += 32) {
+      const double d = part_d2[static_cast<int64_t>(pt) * nq + k];
+      const int64_t i = part_idx[static_cast<int64_t>(pt) * nq + k];
+      if (i >= 0 && (d < b || (d == b && (bi < 0 || i < bi)))) {
+        b = d;
+        bi = i;
+      }
+    }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (acc < best) {  // j increases, so the first minimum is kept
-        best = acc;
-        bidx = j;
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ob = __shfl_xor_sync(0xffffffffu, b, o);
+      const int64_t oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi >= 0 && (bi < 0 || ob < b || (ob == b && oi < bi))) {
+        b = ob;
+        bi = oi;
       }
     }
     if (lane == 0) {
-      w_best[warp] = best;
-      w_idx[warp] = bidx;
+      s_bd[k] = b;
+      s_bi[k] = static_cast<int>(bi);
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      double b = INFINITY;
-      int bi = 0x7fffffff;
-      for (int w = 0; w < nwarps; ++w) {
-        if (w_best[w] < b || (w_best[w] == b && w_idx[w] < bi)) {
-          b = w_best[w];
-          bi = w_idx[w];
-        }
-      }
-      if (bi == 0x7fffffff) bi = -1;
-      if (argmin) argmin[qi] = bi;
-      if (min_d2) min_d2[qi] = b;
-      const int doit = (cnt > 0 && b > thr2 && s_app < cap && cnt < capacity) ? 1 : 0;
-      s_do_append = doit;
-      if (appended) appended[qi] = static_cast<uint8_t>(doit);
-    }
-    __syncthreads();
-    if (s_do_append) {
-      float* dst = bank + static_cast<int64_t>(cnt) * dim;
-      for (int d = threadIdx.x; d < dim; d += kBankThreads) dst[d] = q[d];
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        s_cnt = cnt + 1;
-        s_app = s_app + 1;
-        if (st && s_app < 4) st->anchor_fire[s_app] = 1;
-      }
-    }
-    __syncthreads();
   }
+  // query-query distances (i < k)
+  for (int p = warp; p < nq * nq; p += nwarps) {
+    const int k = p / nq, i = p - (p / nq) * nq;
+    if (i >= k) continue;   // warp-uniform
+    const double d = dist2_warp(queries + static_cast<int64_t>(k) * dim,
+                                queries + static_cast<int64_t>(i) * dim, dim, lane);
+    if (lane == 0) s_dq[k * kBankMaxQueries + i] = d;
+  }
+  __syncthreads();
   if (threadIdx.x == 0) {
-    if (count_p) *count_p = s_cnt;
-    if (appends_p) *appends_p = s_app;
+    const int n_app = bank_decide(s_bd, s_bi, s_dq, kBankMaxQueries, nq, s_cnt0, s_app0, capacity,
+                                  thr2, cap, argmin, min_d2, appended, s_list, nullptr);
+    s_napp = n_app;
+    *count_p = s_cnt0 + n_app;
+    *appends_p = s_app0 + n_app;
+  }
+  __syncthreads();
+  for (int a = 0; a < s_napp; ++a) {
+    const float* src = queries + static_cast<int64_t>(s_list[a]) * dim;
+    float* dst = bank + static_cast<int64_t>(s_cnt0 + a) * dim;
+    for (int d = threadIdx.x; d < dim; d += kBankThreads) dst[d] = src[d];
+  }
+}
+
+// Nearest of `count` stored vectors to one query (pose retrieval), one CTA.
+__global__ void __launch_bounds__(kBankThreads) nearest_small_kernel(
+    const float* __restrict__ store, int count, int dim, const float* __restrict__ query,
+    int32_t* argmin, double* min_d2) {
+  __shared__ double w_best[kBankThreads / 32];
+  __shared__ int w_idx[kBankThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  double best = INFINITY;
+  int bidx = -1;
+  for (int j = warp; j < count; j += kBankThreads / 32) {
+    const double d = dist2_warp(query, store + static_cast<int64_t>(j) * dim, dim, lane);
+    if (d < best) {   // a warp's entries increase
+      best = d;
+      bidx = j;
+    }
+  }
+  if (lane == 0) {
+    w_best[warp] = best;
+    w_idx[warp] = bidx;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double b = INFINITY;
+    int bi = -1;
+    for (int w = 0; w < kBankThreads / 32; ++w)
+      if (w_idx[w] >= 0 && (w_best[w] < b || (w_best[w] == b && w_idx[w] < bi))) {
+        b = w_best[w];
+        bi = w_idx[w];
+      }
+    *argmin = bi;
+    if (min_d2) *min_d2 = b;
   }
 }
 
@@ -652,23 +971,52 @@ cudaError_t launch_ring_commit(DevState* st, int sessions, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+int bank_parts(int64_t capacity) {
+  constexpr int kEntriesPerCta = kBankThreads / kBankLanes * kBankE;
+  int64_t g = (capacity + kEntriesPerCta - 1) / kEntriesPerCta;
+  if (g > 148 * 8) g = 148 * 8;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+bool bank_small(int capacity, int nq) { return capacity <= kBankSmall && nq <= kBankSmall; }
+
+size_t bank_workspace_bytes(int64_t capacity, int nq) {
+  if (bank_small(static_cast<int>(capacity > 1 << 30 ? 1 << 30 : capacity), nq)) return 0;
+  return static_cast<size_t>(bank_parts(capacity)) * nq * (sizeof(double) + sizeof(int64_t));
+}
+
 cudaError_t launch_bank_check(float* bank, int32_t* count, int32_t* appends, int capacity,
                               int dim, const float* queries, int nq, double thr2, int cap,
                               int32_t* argmin, double* min_d2, uint8_t* appended,
-                              DevState* st, int sessions, cudaStream_t s) {
+                              DevState* st, int sessions, void* workspace, cudaStream_t s) {
   if (!st && sessions != 1) return cudaErrorInvalidValue;
-  bank_check_kernel<<<sessions, kBankThreads, 0, s>>>(bank, count, appends, capacity, dim, queries,
-                                                      nq, thr2, cap, argmin, min_d2, appended, st,
-                                                      0);
+  if (nq < 1 || nq > kBankMaxQueries) return cudaErrorInvalidValue;
+  if (bank_small(capacity, nq)) {
+    bank_check_kernel<<<sessions, kBankThreads, 0, s>>>(bank, count, appends, capacity, dim,
+                                                        queries, nq, thr2, cap, argmin, min_d2,
+                                                        appended, st);
+    return cudaGetLastError();
+  }
+  // large banks: context-free calls only (one session, caller workspace)
+  if (st || !workspace) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(double) * static_cast<size_t>(nq) * dim;
+  if (smem > 160 * 1024) return cudaErrorInvalidValue;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(bank_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return cudaErrorInvalidValue;
+  const int parts = bank_parts(capacity);
+  double* pd = static_cast<double*>(workspace);
+  int64_t* pi = reinterpret_cast<int64_t*>(pd + static_cast<size_t>(parts) * nq);
+  bank_partial_kernel<<<parts, kBankThreads, smem, s>>>(bank, count, capacity, dim, queries, nq, pd,
+                                                        pi);
+  bank_resolve_kernel<<<1, kBankThreads, 0, s>>>(bank, count, appends, capacity, dim, queries, nq,
+                                                 thr2, cap, pd, pi, parts, argmin, min_d2, appended);
   return cudaGetLastError();
 }
-
 cudaError_t launch_nearest(const float* store, int count, int dim, const float* query,
                            int32_t* argmin, double* min_d2, cudaStream_t s) {
-  // a bank check with no append allowed: the nearest stored vector
-  bank_check_kernel<<<1, kBankThreads, 0, s>>>(const_cast<float*>(store), nullptr, nullptr, count,
-                                               dim, query, 1, 0.0, 0, argmin, min_d2, nullptr,
-                                               nullptr, count);
+  nearest_small_kernel<<<1, kBankThreads, 0, s>>>(store, count, dim, query, argmin, min_d2);
   return cudaGetLastError();
 }
 

@@ -52,12 +52,16 @@ cudaError_t launch_ring_push(DevState* st, float* ring, float* slot_motion, floa
 cudaError_t launch_ddim(DevState* st, float* ring, const float* eps, float* out_x0,
                         int64_t frame_elems, const DdimCoef& coef, int sessions, cudaStream_t s);
 cudaError_t launch_ring_commit(DevState* st, int sessions, cudaStream_t s);
-// With st != null the counts live in st[session] and `count`/`appends` are
-// ignored; without it (a standalone bank) sessions must be 1.
+// In-order motion-bank check. With st != null the counts live in st[session]
+// and `count`/`appends` are ignored (capacity and queries <= 32: the one-CTA
+// path); without it (a standalone bank) sessions must be 1, and banks past 32
+// entries or 32 queries take the multi-CTA path, which needs a device
+// workspace of bank_workspace_bytes() (0 for the one-CTA path). nq <= 64.
+size_t bank_workspace_bytes(int64_t capacity, int nq);
 cudaError_t launch_bank_check(float* bank, int32_t* count, int32_t* appends, int capacity,
                               int dim, const float* queries, int nq, double thr2, int cap,
                               int32_t* argmin, double* min_d2, uint8_t* appended,
-                              DevState* st, int sessions, cudaStream_t s);
+                              DevState* st, int sessions, void* workspace, cudaStream_t s);
 // argmin_j ||query - store_j||^2 over `count` stored vectors (fp64, lowest index on ties).
 cudaError_t launch_nearest(const float* store, int count, int dim, const float* query,
                            int32_t* argmin, double* min_d2, cudaStream_t s);

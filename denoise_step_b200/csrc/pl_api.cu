@@ -99,8 +99,12 @@ struct pl_ctx {
   float* slot_motion;
   float* batch_motion;
   float* bank;
+  int motion_blocks;   // motion cross-attention blocks per layer (1 or 2)
   __half* bank_kv[PL_MAX_LAYERS];     // fp16 [S][capacity][N][2C]
   float* motion_kv[PL_MAX_LAYERS];   // fp32 [S][16][32][2C]
+  float* motion_kv2[PL_MAX_LAYERS];  // second motion block's, as motion_kv
+  __half* w_oq[PL_MAX_LAYERS];        // fp16 [C][C] = Wo Mq
+  __half* w_oq2[PL_MAX_LAYERS];       // fp16 [C][C] = Mo Mq2 (two motion blocks)
   __half* qkv;
   __half* attn_o;
   __half* a1;
@@ -143,6 +147,7 @@ size_t layout(const pl_config& c, pl_ctx* ctx) {
   };
   const int capacity = 1 + c.append_cap;
   const int64_t S = c.sessions > 0 ? c.sessions : 1;
+  const bool two = c.motion_blocks == 2;
   const int64_t fe = static_cast<int64_t>(c.latent_c) * c.latent_h * c.latent_w;
   uint8_t* st = take(sizeof(pl::DevState) * S);
   uint8_t* ring = take(sizeof(float) * S * 16 * fe);
@@ -154,9 +159,15 @@ size_t layout(const pl_config& c, pl_ctx* ctx) {
     const int64_t N = c.layer_tokens[l], C = c.layer_channels[l];
     uint8_t* bkv = take(sizeof(__half) * S * capacity * N * 2 * C);
     uint8_t* mkv = take(sizeof(float) * S * 16 * 32 * 2 * C);
+    uint8_t* mkv2 = two ? take(sizeof(float) * S * 16 * 32 * 2 * C) : nullptr;
+    uint8_t* woq = take(sizeof(__half) * C * C);
+    uint8_t* woq2 = two ? take(sizeof(__half) * C * C) : nullptr;
     if (ctx) {
       ctx->bank_kv[l] = reinterpret_cast<__half*>(bkv);
       ctx->motion_kv[l] = reinterpret_cast<float*>(mkv);
+      ctx->motion_kv2[l] = reinterpret_cast<float*>(mkv2);
+      ctx->w_oq[l] = reinterpret_cast<__half*>(woq);
+      ctx->w_oq2[l] = reinterpret_cast<__half*>(woq2);
     }
     if (S * 16 * N * C > max_nc) max_nc = S * 16 * N * C;
   }
@@ -191,6 +202,7 @@ pl_status validate_config(const pl_config* c) {
   if (c->append_cap < 0 || c->append_cap > PL_MAX_BANK - 1) return PL_EINVAL;
   if (!(c->drift_threshold >= 0.f) || !std::isfinite(c->drift_threshold)) return PL_EINVAL;
   if (c->sessions < 0 || c->sessions > kMaxSessions) return PL_EINVAL;
+  if (c->motion_blocks < 0 || c->motion_blocks > 2) return PL_EINVAL;
   for (int l = 0; l < c->n_layers; ++l) {
     const int N = c->layer_tokens[l], C = c->layer_channels[l];
     if (N < 1 || C < 1 || C % c->heads || C % 16) return PL_EINVAL;
@@ -252,6 +264,7 @@ struct RoundArgs {
   float* out_frames;
   uint8_t* appended;
   void* const* layer_out;
+  void* const* attn_out;
 };
 
 // Enqueue one whole round on `s` (also used under stream capture).
@@ -271,6 +284,11 @@ pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
     r = from_cuda(pl::launch_motion_kv(ctx->batch_motion, static_cast<const __half*>(w.m_kv), F,
                                        C, ctx->motion_kv[l], s));
     if (r) return r;
+    if (ctx->motion_blocks == 2) {
+      r = from_cuda(pl::launch_motion_kv(ctx->batch_motion, static_cast<const __half*>(w.m2_kv),
+                                         F, C, ctx->motion_kv2[l], s));
+      if (r) return r;
+    }
     r = single_gemm(a.hidden[l], C, w.w_qkv, 3 * C, ctx->qkv, 3 * C, static_cast<int>(M), 3 * C,
                     C, &ctx->st->status, s);
     if (r) return r;
@@ -299,15 +317,38 @@ pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
     ap.status = &ctx->st->status;
     ar = pl::attn_launch(ap, hd, s);
     if (ar) return ar == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
-    r = single_gemm(ctx->attn_o, C, w.w_o, C, ctx->a1, C, static_cast<int>(M), C, C,
-                    &ctx->st->status, s);
-    if (r) return r;
-    r = single_gemm(ctx->a1, C, w.m_q, C, ctx->qm, C, static_cast<int>(M), C, C,
-                    &ctx->st->status, s, /*out_f32=*/true);
+    uint32_t* status = &ctx->st->status;
+    const int Mi = static_cast<int>(M);
+    if (a.attn_out) {
+      // the sub-layer output is wanted: O Wo, then its motion queries
+      __half* a1 = static_cast<__half*>(a.attn_out[l]);
+      r = single_gemm(ctx->attn_o, C, w.w_o, C, a1, C, Mi, C, C, status, s);
+      if (r) return r;
+      r = single_gemm(a1, C, w.m_q, C, ctx->qm, C, Mi, C, C, status, s, /*out_f32=*/true);
+    } else {
+      // motion queries straight from O: O (Wo Mq)
+      r = single_gemm(ctx->attn_o, C, ctx->w_oq[l], C, ctx->qm, C, Mi, C, C, status, s,
+                      /*out_f32=*/true);
+    }
     if (r) return r;
     r = from_cuda(pl::launch_motion_attn(ctx->qm, C, ctx->motion_kv[l], F, N, C, H, ctx->om, C, s));
     if (r) return r;
-    r = single_gemm(ctx->om, C, w.m_o, C, out, C, static_cast<int>(M), C, C, &ctx->st->status, s);
+    if (ctx->motion_blocks == 2) {
+      // block 2's queries from block 1's output: y1 Mq2 = om (Mo Mq2)
+      if (a.attn_out) {
+        r = single_gemm(ctx->om, C, w.m_o, C, ctx->a1, C, Mi, C, C, status, s);
+        if (r) return r;
+        r = single_gemm(ctx->a1, C, w.m2_q, C, ctx->qm, C, Mi, C, C, status, s, true);
+      } else {
+        r = single_gemm(ctx->om, C, ctx->w_oq2[l], C, ctx->qm, C, Mi, C, C, status, s, true);
+      }
+      if (r) return r;
+      r = from_cuda(pl::launch_motion_attn(ctx->qm, C, ctx->motion_kv2[l], F, N, C, H, ctx->om,
+                                           C, s));
+      if (r) return r;
+    }
+    const void* w_last = ctx->motion_blocks == 2 ? w.m2_o : w.m_o;
+    r = single_gemm(ctx->om, C, w_last, C, out, C, Mi, C, C, status, s);
     if (r) return r;
   }
   r = from_cuda(pl::launch_ddim(ctx->st, ctx->ring, a.eps, a.out_frames, ctx->frame_elems,
@@ -318,7 +359,8 @@ pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
   r = from_cuda(pl::launch_bank_check(ctx->bank, nullptr, nullptr, ctx->capacity, 512,
                                       a.new_motion, 4,
                                       static_cast<double>(c.drift_threshold) * c.drift_threshold,
-                                      c.append_cap, nullptr, nullptr, a.appended, ctx->st, S, s));
+                                      c.append_cap, nullptr, nullptr, a.appended, ctx->st, S,
+                                      nullptr, s));
   if (r) return r;
   if (ctx->have_anchors) {
     for (int an = 1; an <= c.append_cap; ++an) {
@@ -394,7 +436,7 @@ const char* pl_status_string(int status) {
   }
 }
 
-int pl_abi_version(void) { return 1; }
+int pl_abi_version(void) { return 2; }
 
 pl_status pl_gemm_f16(const void* a, int64_t lda, const void* b, int64_t ldb, void* c,
                       int64_t ldc, int M, int N, int K, void* stream) {
@@ -599,18 +641,34 @@ pl_status pl_motion_xattn(const void* x, const float* motion, const void* m_q, c
   return single_gemm(om, c, m_o, c, out, c, frames * n, c, c, status, s);
 }
 
+pl_status pl_motion_bank_check_workspace_bytes(int capacity, int dim, int n_queries,
+                                               size_t* bytes) {
+  if (!bytes || capacity < 1 || capacity > (1 << 24) || dim < 1 || dim > 4096) return PL_EINVAL;
+  if (n_queries < 0 || n_queries > 64) return PL_EINVAL;
+  *bytes = n_queries == 0 ? 0 : pl::bank_workspace_bytes(capacity, n_queries);
+  return PL_OK;
+}
+
 pl_status pl_motion_bank_check(float* bank, int32_t* count, int32_t* appends, int capacity,
                                int dim, const float* queries, int n_queries, float threshold,
                                int cap, int32_t* argmin, double* min_d2, uint8_t* appended,
-                               void* stream) {
+                               void* workspace, size_t workspace_bytes, void* stream) {
   if (!bank || !count || !appends || (n_queries > 0 && !queries)) return PL_EINVAL;
-  if (dim < 1 || dim > 4096 || capacity < 1 || capacity > 65536) return PL_EINVAL;
+  if (dim < 1 || dim > 4096 || capacity < 1 || capacity > (1 << 24)) return PL_EINVAL;
   if (n_queries < 0 || n_queries > 64 || cap < 0) return PL_EINVAL;
   if (!(threshold >= 0.f) || !std::isfinite(threshold)) return PL_EINVAL;
   if (n_queries == 0) return PL_OK;
+  size_t need = 0;
+  if (pl_motion_bank_check_workspace_bytes(capacity, dim, n_queries, &need)) return PL_EINVAL;
+  if (need > 0) {
+    if (!workspace || !aligned16(workspace)) return PL_EINVAL;
+    if (workspace_bytes < need) return PL_ENOMEM;
+    if (static_cast<size_t>(n_queries) * dim * sizeof(double) > 160 * 1024) return PL_EUNSUPPORTED;
+  }
   const double thr2 = static_cast<double>(threshold) * threshold;
   return from_cuda(pl::launch_bank_check(bank, count, appends, capacity, dim, queries, n_queries,
                                          thr2, cap, argmin, min_d2, appended, nullptr, 1,
+                                         need > 0 ? workspace : nullptr,
                                          static_cast<cudaStream_t>(stream)));
 }
 
@@ -662,6 +720,7 @@ pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_
   ctx->cfg = *cfg;
   ctx->sessions = cfg->sessions > 0 ? cfg->sessions : 1;
   ctx->capacity = 1 + cfg->append_cap;
+  ctx->motion_blocks = cfg->motion_blocks == 2 ? 2 : 1;
   ctx->frame_elems = static_cast<int64_t>(cfg->latent_c) * cfg->latent_h * cfg->latent_w;
   ctx->ws = static_cast<uint8_t*>(workspace);
   ctx->ws_bytes = workspace_bytes;
@@ -708,6 +767,7 @@ pl_status pl_bank_init(pl_ctx* ctx, const pl_layer_weights* weights,
   for (int l = 0; l < L; ++l) {
     const pl_layer_weights& w = weights[l];
     if (!w.w_qkv || !w.w_o || !w.m_q || !w.m_kv || !w.m_o || !ref_feats[l]) return PL_EINVAL;
+    if (ctx->motion_blocks == 2 && (!w.m2_q || !w.m2_kv || !w.m2_o)) return PL_EINVAL;
     ctx->w[l] = w;
     ctx->ref_feats[l] = ref_feats[l];
   }
@@ -728,6 +788,17 @@ pl_status pl_bank_init(pl_ctx* ctx, const pl_layer_weights* weights,
   if (L > 0) {
     r = project_bank(ctx, ctx->ref_feats, 0, /*predicated=*/false, s);
     if (r) return r;
+  }
+  // the folded projections Wo Mq (and Mo Mq2), fp32 accumulation, one rounding
+  for (int l = 0; l < L; ++l) {
+    const int C = ctx->cfg.layer_channels[l];
+    const pl_layer_weights& w = ctx->w[l];
+    r = single_gemm(w.w_o, C, w.m_q, C, ctx->w_oq[l], C, C, C, C, &ctx->st->status, s);
+    if (r) return r;
+    if (ctx->motion_blocks == 2) {
+      r = single_gemm(w.m_o, C, w.m2_q, C, ctx->w_oq2[l], C, C, C, C, &ctx->st->status, s);
+      if (r) return r;
+    }
   }
   ctx->initialised = true;
   return PL_OK;
@@ -763,7 +834,7 @@ pl_status pl_ctx_bank_check(pl_ctx* ctx, const float* queries, int n_queries, in
   pl_status r = from_cuda(pl::launch_bank_check(
       ctx->bank, nullptr, nullptr, ctx->capacity, 512, queries, n_queries,
       static_cast<double>(c.drift_threshold) * c.drift_threshold, c.append_cap, argmin, min_d2,
-      appended, ctx->st, ctx->sessions, s));
+      appended, ctx->st, ctx->sessions, nullptr, s));
   if (r) return r;
   if (ctx->have_anchors) {
     for (int an = 1; an <= c.append_cap; ++an) {
@@ -776,7 +847,8 @@ pl_status pl_ctx_bank_check(pl_ctx* ctx, const float* queries, int n_queries, in
 
 pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_motion,
                           const void* const* hidden, const float* eps, float* out_frames,
-                          uint8_t* appended, void* const* layer_out, void* stream) {
+                          uint8_t* appended, void* const* layer_out, void* const* attn_out,
+                          void* stream) {
   if (!ctx || !new_noise || !new_motion || !eps || !out_frames) return PL_EINVAL;
   if (!ctx->initialised) return PL_ESTATE;
   const int L = ctx->cfg.n_layers;
@@ -784,14 +856,16 @@ pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_
   for (int l = 0; l < L; ++l) {
     if (!hidden[l] || !aligned16(hidden[l])) return PL_EINVAL;
     if (layer_out && (!layer_out[l] || !aligned16(layer_out[l]))) return PL_EINVAL;
+    if (attn_out && (!attn_out[l] || !aligned16(attn_out[l]))) return PL_EINVAL;
   }
   if (!aligned16(new_noise) || !aligned16(eps) || !aligned16(out_frames)) return PL_EINVAL;
-  RoundArgs a{new_noise, new_motion, hidden, eps, out_frames, appended, layer_out};
+  RoundArgs a{new_noise, new_motion, hidden, eps, out_frames, appended, layer_out, attn_out};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const char* env = std::getenv("PL_NO_GRAPH");
   const bool use_graph = s != nullptr && !(env && env[0] == '1');
   if (!use_graph) return enqueue_round(ctx, a, s);
   // key = every pointer the captured launches bake in
+  static_assert(7 + 3 * PL_MAX_LAYERS <= 64, "graph key size");
   const void* key[64];
   int kn = 0;
   key[kn++] = new_noise;
@@ -800,9 +874,11 @@ pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_
   key[kn++] = out_frames;
   key[kn++] = appended;
   key[kn++] = layer_out ? reinterpret_cast<const void*>(1) : nullptr;
+  key[kn++] = attn_out ? reinterpret_cast<const void*>(1) : nullptr;
   for (int l = 0; l < L; ++l) {
     key[kn++] = hidden[l];
     key[kn++] = layer_out ? layer_out[l] : nullptr;
+    key[kn++] = attn_out ? attn_out[l] : nullptr;
   }
   pl_ctx::GraphSlot* slot = nullptr;
   for (auto& g : ctx->graphs) {
@@ -891,7 +967,7 @@ pl_status pl_stream_round_host(pl_ctx* ctx, void* staging, size_t staging_bytes,
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ctx->ev_in[b], 0);
   if (e != cudaSuccess) return PL_ECUDA;
   const pl_status r = pl_stream_round(ctx, h.noise, h.motion, h.hidden, h.eps, h.out, nullptr,
-                                      nullptr, stream);
+                                      nullptr, nullptr, stream);
   if (r != PL_OK) return r;
   if (cudaEventRecord(ctx->ev_free[b], s) != cudaSuccess) return PL_ECUDA;
   ctx->free_pending[b] = true;

@@ -6,6 +6,7 @@
     python -m denoise_step_b200.microbench sink --n 4096 --c 5120 --heads 40 --pool 64 --reps 3
     python -m denoise_step_b200.microbench nearest --count 1048576 --dim 128 --reps 10
     python -m denoise_step_b200.microbench motion --frames 16 --n 4096 --c 320 --heads 8 --reps 10
+    python -m denoise_step_b200.microbench bank --count 4 --dim 512 --queries 4 --reps 10
 
 Inputs are seeded torch tensors on the device; prints the mean CUDA-event time
 per launch and the algorithmic throughput.
@@ -128,9 +129,25 @@ def ddim(a, stream):
     return {"kernel": "ring push + ddim", "s": t, "gbs_ddim_bytes": byts / t / 1e9}
 
 
+def bank(a, stream):
+    """Motion-bank check: `queries` N(0, 4) embeddings checked in order against
+    `count` stored N(0, 4) vectors of `dim` (no room to append, so every call
+    does the same work); algorithmic bytes = (count + queries) * dim * 4."""
+    g = torch.Generator(device="cuda").manual_seed(a.seed)
+    store = 2.0 * torch.randn((a.count, a.dim), device="cuda", generator=g)
+    qs = 2.0 * torch.randn((a.queries, a.dim), device="cuda", generator=g)
+    cnt = torch.full((1,), a.count, dtype=torch.int32, device="cuda")
+    app = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fn = lambda: P.motion_bank_check(store, cnt, app, qs, 17.0, 3, stream=stream)
+    t = _time(fn, a.reps, stream)
+    return {"kernel": "bank check", "s": t, "us": t * 1e6,
+            "gbs": 4.0 * (a.count + a.queries) * a.dim / t / 1e9}
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["attn", "gemm", "ddim", "sink", "nearest", "motion"])
+    ap.add_argument("what", choices=["attn", "gemm", "ddim", "sink", "nearest", "motion", "bank"])
+    ap.add_argument("--queries", type=int, default=4)
     ap.add_argument("--count", type=int, default=1 << 20)
     ap.add_argument("--dim", type=int, default=128)
     ap.add_argument("--pool", type=int, default=64)
@@ -148,7 +165,7 @@ def main():
     a = ap.parse_args()
     stream = torch.cuda.Stream()
     r = {"attn": attn, "gemm": gemm, "ddim": ddim, "sink": sink, "nearest": nearest,
-         "motion": motion}[a.what](a, stream)
+         "motion": motion, "bank": bank}[a.what](a, stream)
     print(json.dumps(r))
 
 

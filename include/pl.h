@@ -201,11 +201,18 @@ pl_status pl_motion_xattn(const void* x, const float* motion, const void* m_q,
  * argmin (int32), min_d2 (double), appended (uint8): device [n_queries],
  * each may be NULL. cap = 0 turns the call into a pure nearest-neighbour
  * retrieval (LiveAnimate page, PR-Sink's pose-retrieved dynamic sink).
- * 1 <= dim <= 4096, 1 <= capacity <= 65536, 0 <= n_queries <= 64. */
+ * 1 <= dim <= 4096, 1 <= capacity <= 2^24, 0 <= n_queries <= 64.
+ * Banks of up to 32 entries checked with up to 32 queries run in one CTA
+ * and need no workspace (workspace may be NULL). Larger ones read the bank
+ * once for all queries across the GPU and keep per-CTA minima in a device
+ * workspace of pl_motion_bank_check_workspace_bytes() (16-byte aligned;
+ * PL_ENOMEM when smaller); they also need n_queries * dim <= 20480. */
+pl_status pl_motion_bank_check_workspace_bytes(int capacity, int dim, int n_queries,
+                                               size_t* bytes);
 pl_status pl_motion_bank_check(float* bank, int32_t* count, int32_t* appends, int capacity,
                                int dim, const float* queries, int n_queries, float threshold,
                                int cap, int32_t* argmin, double* min_d2, uint8_t* appended,
-                               void* stream);
+                               void* workspace, size_t workspace_bytes, void* stream);
 
 /* Bytes of device workspace pl_nearest needs for a store of `count` entries. */
 pl_status pl_nearest_workspace_bytes(int64_t count, size_t* bytes);
@@ -395,6 +402,13 @@ typedef struct pl_config {
   int32_t append_cap;                    /* 3 (so the bank holds at most 4) */
   int32_t sessions;                      /* independent streams served together, 1..8
                                             (0 is read as 1); see below */
+  int32_t motion_blocks;                 /* motion cross-attention blocks per layer:
+                                            1 (0 is read as 1) or 2 (PersonaLive
+                                            write-up, "三条条件通路": the motion
+                                            module's attention blocks are
+                                            [Spatial_Cross, Spatial_Cross]; block 2
+                                            has its own weights, the same 32 tokens,
+                                            and block 1's output as its queries) */
 } pl_config;
 
 /* Sessions. A context serves S = cfg.sessions independent streams (same
@@ -412,6 +426,9 @@ typedef struct pl_layer_weights {
   const void* m_q;   /* [C][C] motion query projection */
   const void* m_kv;  /* [16][2C] = [Mk | Mv] */
   const void* m_o;   /* [C][C] */
+  const void* m2_q;  /* second motion block (motion_blocks == 2, else NULL): [C][C] */
+  const void* m2_kv; /* [16][2C] */
+  const void* m2_o;  /* [C][C] */
 } pl_layer_weights;
 
 /* Host-side snapshot of the context's state (pl_get_state). */
@@ -442,6 +459,10 @@ pl_status pl_ctx_destroy(pl_ctx* ctx);
 /* Reference fusion, also the control-plane reset (PersonaLive write-up,
  * "首帧怎么办" and the pause/reset remark of "在线链路"):
  *  - KV bank <- entry 0 = ref_feats[l] projected by each layer's Wk/Wv;
+ *  - per layer, the products Wo Mq (and Mo Mq2 with two motion blocks),
+ *    accumulated in fp32 and rounded once to fp16: no nonlinearity sits
+ *    between the O projection and the next motion query projection, so the
+ *    round applies them as one [C][C] projection;
  *  - motion bank <- [ref_motion], appends <- 0;
  *  - prefill: 3 windows at t = 0, 333, 666 (oldest first), window w frame j =
  *    sqrt(abar_t) ref_latent + sqrt(1 - abar_t) prefill_eps[4w + j], with the
@@ -483,12 +504,17 @@ pl_status pl_ctx_bank_check(pl_ctx* ctx, const float* queries, int n_queries,
  * hidden: host array [n_layers] of device fp16 [16][N_l][C_l] (batch order);
  * eps: device fp32 [16][4][H][W]; out_frames: device fp32 [4][4][H][W];
  * appended: device uint8 [4] or NULL; layer_out: host array [n_layers] of
- * device fp16 [16][N_l][C_l] or NULL (outputs then go to workspace).
+ * device fp16 [16][N_l][C_l] or NULL (outputs then go to workspace);
+ * attn_out: host array [n_layers] of device fp16 [16][N_l][C_l] or NULL:
+ * when given, each layer's reference-attention sub-layer output (before the
+ * motion cross-attention) is written there, and the round then applies Wo
+ * and Mq (and Mo, Mq2) as separate projections instead of their products.
  * The round is recorded as a CUDA graph on the first call and replayed while
  * the pointer arguments stay the same. */
 pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_motion,
                           const void* const* hidden, const float* eps, float* out_frames,
-                          uint8_t* appended, void* const* layer_out, void* stream);
+                          uint8_t* appended, void* const* layer_out,
+                          void* const* attn_out, void* stream);
 
 /* Host-buffer round: the serving boundary of the PersonaLive write-up,
  * "在线链路" (frames arrive from the host, four at a time, one forward per

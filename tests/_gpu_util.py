@@ -22,14 +22,20 @@ def layer_weights_np(seed, name, C):
 
 
 def pack_weights(w):
-    """Device tensors in the library's layout: w_qkv = [Wq|Wk|Wv], m_kv = [Mk|Mv]."""
-    return {
+    """Device tensors in the library's layout: w_qkv = [Wq|Wk|Wv], m_kv = [Mk|Mv]
+    (and m2_* for a second motion block when w holds mq2, mk2, mv2, mo2)."""
+    out = {
         "w_qkv": dev(np.concatenate([w["wq"], w["wk"], w["wv"]], axis=1)),
         "w_o": dev(w["wo"]),
         "m_q": dev(w["mq"]),
         "m_kv": dev(np.concatenate([w["mk"], w["mv"]], axis=1)),
         "m_o": dev(w["mo"]),
     }
+    if "mq2" in w:
+        out["m2_q"] = dev(w["mq2"])
+        out["m2_kv"] = dev(np.concatenate([w["mk2"], w["mv2"]], axis=1))
+        out["m2_o"] = dev(w["mo2"])
+    return out
 
 
 def attn_errors(got, want):

@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings_and_abi():
     import denoise_step_b200 as P
-    assert P.lib.pl_abi_version() == 1
+    assert P.lib.pl_abi_version() == 2
     for s in range(8):
         assert P.lib.pl_status_string(s)
     assert P.lib.pl_status_string(99) == b"unknown status"
@@ -50,7 +50,15 @@ def test_host_validation_rejects_bad_arguments():
     seg = (P.KVSegment * 1)()
     assert L.pl_segment_attention(None, 8, 8, seg, 1, 1, 1, 1, 40, None, 8, 8, None) == P.PL_EINVAL
     assert L.pl_motion_bank_check(None, None, None, 4, 512, None, 1, 17.0, 3, None, None, None,
-                                  None) == P.PL_EINVAL
+                                  None, 0, None) == P.PL_EINVAL
+    # the one-CTA check needs no workspace; larger banks need per-CTA minima
+    assert L.pl_motion_bank_check_workspace_bytes(32, 512, 32, C.byref(n)) == P.PL_OK
+    assert n.value == 0
+    assert L.pl_motion_bank_check_workspace_bytes(33, 512, 4, C.byref(n)) == P.PL_OK
+    assert n.value >= 16 * 4
+    assert L.pl_motion_bank_check_workspace_bytes(4, 512, 33, C.byref(n)) == P.PL_OK
+    assert n.value >= 16 * 33
+    assert L.pl_motion_bank_check_workspace_bytes(4, 512, 65, C.byref(n)) == P.PL_EINVAL
     assert L.pl_ctx_destroy(None) == P.PL_OK
 
 
@@ -84,12 +92,29 @@ def test_sessions_scale_the_workspace():
         assert P.lib.pl_workspace_bytes(C.byref(cfg), C.byref(n)) == P.PL_OK
         sizes[sess] = n.value
     assert sizes[0] == sizes[1]                        # 0 is read as one session
-    # every buffer is per session (256-byte rounding aside)
-    assert abs(sizes[2] - 2 * sizes[1]) < 64 * 256
-    assert abs(sizes[8] - 8 * sizes[1]) < 256 * 256
+    # every buffer is per session except the folded [C][C] projections
+    # (Wo Mq per layer, fp16), which all sessions share (256-byte rounding aside)
+    shared = sum(2 * c * c for _, c in layers)
+    assert abs(sizes[2] - 2 * sizes[1] + shared) < 64 * 256
+    assert abs(sizes[8] - 8 * sizes[1] + 7 * shared) < 256 * 256
     for sess in (-1, 9):
         cfg = P.make_config((64, 64), layers, sessions=sess)
         assert P.lib.pl_workspace_bytes(C.byref(cfg), C.byref(n)) == P.PL_EINVAL
+
+
+def test_second_motion_block_adds_its_buffers():
+    import denoise_step_b200 as P
+    import synthetic as S
+    layers = [(side * side, c) for _, side, c in S.LAYERS]
+    n1, n2 = C.c_size_t(), C.c_size_t()
+    for blocks, n in ((1, n1), (2, n2)):
+        cfg = P.make_config((64, 64), layers, motion_blocks=blocks)
+        assert P.lib.pl_workspace_bytes(C.byref(cfg), C.byref(n)) == P.PL_OK
+    # per layer: the block's motion K/V (fp32 [16][32][2C]) and Mo Mq2 (fp16 [C][C])
+    extra = sum(4 * 16 * 32 * 2 * c + 2 * c * c for _, c in layers)
+    assert abs(n2.value - n1.value - extra) < 64 * 256
+    bad = P.make_config((64, 64), layers, motion_blocks=3)
+    assert P.lib.pl_workspace_bytes(C.byref(bad), C.byref(n1)) == P.PL_EINVAL
 
 
 def test_host_staging_size_and_validation():
@@ -118,7 +143,8 @@ def test_host_staging_size_and_validation():
 def test_round_before_init_is_a_state_error():
     import denoise_step_b200 as P
     # a null context is rejected before any device work
-    assert P.lib.pl_stream_round(None, None, None, None, None, None, None, None, None) == P.PL_EINVAL
+    assert P.lib.pl_stream_round(None, None, None, None, None, None, None, None, None,
+                                 None) == P.PL_EINVAL
     assert P.lib.pl_ring_push(None, None, None, None) == P.PL_EINVAL
 
 

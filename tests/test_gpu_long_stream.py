@@ -2,7 +2,10 @@
 
 Every round: x0 frames within 1e-5, append flags and the pile / bank state
 bit-exact. Attention is spot-checked on rounds 1, 2, 3, 4, 100 and 3600 (one
-layer per level, sampled rows). The 512-d motion embedding follows a seeded
+layer per level, sampled rows). On rounds 1, 100 and 3600 the round also
+returns each layer's reference-attention sub-layer output, which is held to
+the plain attention gates (max abs 1e-2, mean abs 1e-3, no scaling); those
+rounds apply Wo and Mq separately, the others their folded product. The 512-d motion embedding follows a seeded
 Gaussian random walk with step sigma 3, so the cap of 3 appends is reached in
 round 1 and the state then stays constant: 4 frames in, 4 out, forever.
 """
@@ -21,6 +24,7 @@ torch = pytest.importorskip("torch")
 
 ROUNDS = 3600
 SPOT = {1, 2, 3, 4, 100, ROUNDS}
+SUBLAYER = {1, 100, ROUNDS}
 
 
 def _motion_logit_std(h, w, bank, motion, rows, heads=8):
@@ -63,6 +67,7 @@ def test_long_stream_3600_rounds():
     out = torch.empty((4, 4, 64, 64), dtype=torch.float32, device="cuda")
     flags = torch.zeros(4, dtype=torch.uint8, device="cuda")
     layer_out = [torch.empty((16, s * s, C), dtype=torch.float16, device="cuda") for _, s, C in L]
+    attn_out = [torch.empty((16, s * s, C), dtype=torch.float16, device="cuda") for _, s, C in L]
     mot_dev = torch.empty((4, 512), dtype=torch.float32, device="cuda")
     # fixed round-input buffers, so the recorded round graph is replayed every round
     noise_dev = torch.empty((4, 4, 64, 64), dtype=torch.float32, device="cuda")
@@ -85,7 +90,8 @@ def test_long_stream_3600_rounds():
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             ev[0].record(stream)
-            st.round(noise_dev, mot_dev, d_hidden, eps_dev, out, flags, layer_out, stream=stream)
+            st.round(noise_dev, mot_dev, d_hidden, eps_dev, out, flags, layer_out, stream=stream,
+                     attn_out=attn_out if r in SUBLAYER else None)
             ev[1].record(stream)
         stream.synchronize()
         gpu_ms += ev[0].elapsed_time(ev[1])
@@ -98,7 +104,12 @@ def test_long_stream_3600_rounds():
                 rows = np.unique(rows_all % (side * side))
                 bank = [ref_feats[li]] + [anchors[a][li] for a in range(n_kv - 1)]
                 got = host(layer_out[li])
+                got_a = host(attn_out[li]) if r in SUBLAYER else None
                 for f in (0, 15):
+                    if got_a is not None:
+                        want_a = O.ref_attention_frame(hidden[li][f], w[li], bank, 8, rows=rows)
+                        mx, mean, rel = attn_errors(got_a[f][rows], want_a)
+                        assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (r, li, f, mx, mean, rel)
                     want = O.layer_forward_frame(hidden[li][f], w[li], bank, O.motion_tokens(bm[f]),
                                                  8, rows=rows)
                     mx, mean, rel = attn_errors(got[f][rows], want)

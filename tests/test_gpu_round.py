@@ -163,7 +163,10 @@ def test_host_round_matches_device_round(P):
 
 def test_full_geometry_rounds_spot_checked(P):
     # 16 reference-attention layers in the SD-UNet layout, bank x4 after round 1,
-    # DDIM on 16x4x64x64, bank check; sampled rows of one layer per level
+    # DDIM on 16x4x64x64, bank check; sampled rows of one layer per level. In
+    # round 2 the round also returns the reference-attention sub-layer output
+    # (Wo and Mq then applied separately), held to the plain attention gates;
+    # rounds 1 and 3 run the folded Wo Mq projection
     case = Case(S.SEEDS["full"], list(S.LAYERS), 64, 64, 3.0)
     st, orc, _ = _setup(P, case)
     stream = torch.cuda.Stream()
@@ -171,6 +174,7 @@ def test_full_geometry_rounds_spot_checked(P):
     flags = torch.zeros(4, dtype=torch.uint8, device="cuda")
     layer_out = [torch.empty((16, side * side, C), dtype=torch.float16, device="cuda")
                  for _, side, C in case.layers]
+    attn_out = [torch.empty_like(t) for t in layer_out]
     check_layers = {0: "d00", 2: "d10", 4: "d20", 6: "m", 15: "u32"}
     rows_all = S.uniform_int(case.seed, "rows", 24, 4096)
     for r in range(1, 4):
@@ -180,7 +184,8 @@ def test_full_geometry_rounds_spot_checked(P):
         d_noise, d_mot, d_eps = dev(noise), dev(mot), dev(eps)
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
-            st.round(d_noise, d_mot, d_hidden, d_eps, out, flags, layer_out, stream=stream)
+            st.round(d_noise, d_mot, d_hidden, d_eps, out, flags, layer_out, stream=stream,
+                     attn_out=attn_out if r == 2 else None)
         stream.synchronize()
         n_kv = 1 + orc.appends
         orc.append(noise, mot)
@@ -190,7 +195,13 @@ def test_full_geometry_rounds_spot_checked(P):
             N = side * side
             rows = np.unique(rows_all % N)
             got = host(layer_out[li])
+            got_a = host(attn_out[li]) if r == 2 else None
             for f in (0, 9):
+                if got_a is not None:
+                    want_a = O.ref_attention_frame(hidden[li][f], case.w[li],
+                                                   _kv_bank(case, li, n_kv), 8, rows=rows)
+                    mx, mean, rel = attn_errors(got_a[f][rows], want_a)
+                    assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (r, li, f, mx, mean, rel)
                 want = O.layer_forward_frame(hidden[li][f], case.w[li], _kv_bank(case, li, n_kv),
                                              O.motion_tokens(bm[f]), 8, rows=rows)
                 mx, mean, rel = attn_errors(got[f][rows], want)
@@ -204,4 +215,76 @@ def test_full_geometry_rounds_spot_checked(P):
         s = st.state()
         assert s["appends"] == orc.appends and s["device_status"] == 0
     assert orc.appends == 3
+    st.close()
+
+
+def _block2_logit_std(h, w, bank, motion, heads=8):
+    """Std of the second motion block's logits (fp64, oracle inputs)."""
+    tok = O.motion_tokens(motion)
+    y1 = O.motion_xattn_frame(O.ref_attention_frame(h, w, bank, heads), tok, w, heads)
+    q = y1 @ np.asarray(w["mq2"], np.float64)
+    k = tok @ np.asarray(w["mk2"], np.float64)
+    hd = q.shape[1] // heads
+    s = [q[:, i * hd:(i + 1) * hd] @ k[:, i * hd:(i + 1) * hd].T / np.sqrt(hd) for i in range(heads)]
+    return float(np.std(np.concatenate([x.ravel() for x in s])))
+
+
+@pytest.mark.parametrize("sublayer", [False, True])
+def test_two_motion_blocks_tiny_rounds(P, sublayer):
+    # two motion cross-attention blocks per layer (own weights, same tokens,
+    # block 2 queried by block 1's output), tiny geometry, 3 rounds; with
+    # `sublayer` the round also returns the reference-attention output and
+    # applies Wo, Mq, Mo, Mq2 separately, else their folded products. Block
+    # 2's queries come from block 1's fp16 output, whose magnitude follows the
+    # walking motion embedding, and its softmax multiplies that rounding by
+    # the spread of its logits: the layer-output gates carry that factor
+    # (kappa, as on the long stream); the sub-layer output has plain gates
+    case = Case(S.SEEDS["tiny"] + 7, [("m", 8, 1280)], 8, 8, 3.0)
+    case.w[0].update(S.motion_block_weights(case.seed, "m", 1280, 2, np.float16))
+    cfg = P.make_config((8, 8), [(64, 1280)], motion_blocks=2)
+    st = P.Stream(cfg)
+    pw = [pack_weights(w) for w in case.w]
+    drive0 = S.normal(case.seed, "drive0", (512,), 1.0, np.float32)
+    st.bank_init(pw, [dev(f) for f in case.ref_feats], [dev(a) for an in case.anchors for a in an],
+                 dev(case.ref_motion), dev(drive0), dev(case.ref_latent), dev(case.prefill_eps))
+    orc = O.PyramidStream(case.ref_latent, case.prefill_eps, case.ref_motion, drive0,
+                          state_dtype=np.float32)
+    stream = torch.cuda.Stream()
+    out = torch.empty((4, 4, 8, 8), dtype=torch.float32, device="cuda")
+    flags = torch.zeros(4, dtype=torch.uint8, device="cuda")
+    layer_out = [torch.empty((16, 64, 1280), dtype=torch.float16, device="cuda")]
+    attn_out = [torch.empty_like(layer_out[0])] if sublayer else None
+    for r in range(1, 4):
+        hidden, noise, eps = case.round_inputs(r)
+        mot = case.next_motion(r)
+        d_in = ([dev(h) for h in hidden], dev(noise), dev(mot), dev(eps))
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            st.round(d_in[1], d_in[2], d_in[0], d_in[3], out, flags, layer_out, stream=stream,
+                     attn_out=attn_out)
+        stream.synchronize()
+        n_kv = 1 + orc.appends
+        orc.append(noise, mot)
+        bm = orc.batch_motion()
+        got = host(layer_out[0])
+        for f in range(0, 16, 3):
+            bank = _kv_bank(case, 0, n_kv)
+            want = O.layer_forward_frame(hidden[0][f], case.w[0], bank, O.motion_tokens(bm[f]), 8,
+                                         motion_blocks=2)
+            mx, mean, rel = attn_errors(got[f], want)
+            g = scaled_gates(want)
+            kappa = max(1.0, _block2_logit_std(hidden[0][f], case.w[0], bank, bm[f]))
+            assert mx <= ATTN_MAX_ABS * g * kappa and mean <= ATTN_MEAN_ABS * g * kappa, \
+                (r, f, mx, mean, rel, g, kappa)
+            assert rel < 2e-3 * kappa, (r, f, rel, kappa)
+            if sublayer:
+                want_a = O.ref_attention_frame(hidden[0][f], case.w[0], bank, 8)
+                mx, mean, rel = attn_errors(host(attn_out[0])[f], want_a)
+                assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (r, f, mx, mean, rel)
+        want_x0 = orc.step_and_pop(eps)
+        _, _, want_flags = orc.check_bank(mot)
+        orc.rounds += 1
+        assert np.max(np.abs(host(out) - want_x0)) <= DDIM_ABS, r
+        assert list(host(flags)) == want_flags, r
+    assert st.device_status() == 0
     st.close()
