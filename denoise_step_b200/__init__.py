@@ -116,6 +116,11 @@ _SIGS = {
     "pl_get_motion_bank": (i32, [vp, vp, C.POINTER(C.c_int32), vp]),
     "pl_get_session_motion_bank": (i32, [vp, i32, vp, C.POINTER(C.c_int32), vp]),
     "pl_get_device_status": (i32, [vp, vp]),
+    "pl_set_profiling": (i32, [vp, i32]),
+    "pl_get_layer_ms": (i32, [vp, vp, i32]),
+    "pl_state_bytes": (i32, [vp, C.POINTER(sz)]),
+    "pl_state_export": (i32, [vp, vp, sz, vp]),
+    "pl_state_import": (i32, [vp, vp, sz, vp]),
     "pl_ctx_ring_latents": (vp, [vp]),
     "pl_sink_workspace_bytes": (i32, [i32, i32, i32, i32, i32, C.POINTER(sz)]),
     "pl_sink_create": (i32, [i32, i32, i32, i32, i32, vp, sz, C.POINTER(vp)]),
@@ -483,6 +488,33 @@ class Stream:
 
     def device_status(self, stream=None) -> int:
         return lib.pl_get_device_status(self.handle, _stream(stream))
+
+    def set_profiling(self, on: bool = True):
+        check(lib.pl_set_profiling(self.handle, 1 if on else 0), "pl_set_profiling")
+
+    def layer_ms(self):
+        """Per-layer times (ms) of the latest profiled round."""
+        L = self.cfg.n_layers
+        buf = (C.c_float * max(L, 1))()
+        check(lib.pl_get_layer_ms(self.handle, buf, L), "pl_get_layer_ms")
+        return [buf[i] for i in range(L)]
+
+    def export_state(self, stream=None):
+        """Snapshot of the streams' state as a numpy uint8 array (blocks)."""
+        import numpy as np
+        n = sz()
+        check(lib.pl_state_bytes(self.handle, C.byref(n)), "pl_state_bytes")
+        buf = np.zeros(n.value, dtype=np.uint8)
+        check(lib.pl_state_export(self.handle, buf.ctypes.data, n.value, _stream(stream)),
+              "pl_state_export")
+        return buf
+
+    def import_state(self, snapshot, stream=None):
+        """Restore a snapshot taken by export_state (after bank_init; blocks)."""
+        import numpy as np
+        buf = np.ascontiguousarray(snapshot, dtype=np.uint8)
+        check(lib.pl_state_import(self.handle, buf.ctypes.data, buf.size, _stream(stream)),
+              "pl_state_import")
 
     def ring_latents(self):
         return lib.pl_ctx_ring_latents(self.handle)

@@ -133,6 +133,10 @@ struct pl_ctx {
   cudaEvent_t ev_free[2];   // the round reading set b is done
   bool free_pending[2];
   int64_t host_rounds;
+  // per-layer timing of rounds run outside the captured graph
+  bool profile;
+  bool prof_valid;             // the events hold a finished profiled round
+  cudaEvent_t prof_ev[PL_MAX_LAYERS + 1];
 };
 
 namespace {
@@ -216,8 +220,9 @@ pl_status validate_config(const pl_config* c) {
 // with `predicated` a session's launch only runs when that session's bank
 // check appended anchor `entry` this round.
 pl_status project_bank(pl_ctx* ctx, const void* const* feats, int entry, bool predicated,
-                       cudaStream_t s) {
+                       cudaStream_t s, int only_session = -1) {
   for (int z = 0; z < ctx->sessions; ++z) {
+    if (only_session >= 0 && z != only_session) continue;
     GemmParams gp;
     std::memset(&gp, 0, sizeof(gp));
     gp.status = &ctx->st[z].status;
@@ -265,6 +270,7 @@ struct RoundArgs {
   uint8_t* appended;
   void* const* layer_out;
   void* const* attn_out;
+  cudaEvent_t* layer_events;   // when non-null: [n_layers + 1] recorded around the layers
 };
 
 // Enqueue one whole round on `s` (also used under stream capture).
@@ -277,6 +283,7 @@ pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
                                                ctx->frame_elems, S, s));
   if (r) return r;
   for (int l = 0; l < c.n_layers; ++l) {
+    if (a.layer_events && cudaEventRecord(a.layer_events[l], s) != cudaSuccess) return PL_ECUDA;
     const int N = c.layer_tokens[l], C = c.layer_channels[l], H = c.heads, hd = C / H;
     const int64_t M = static_cast<int64_t>(F) * N;
     const pl_layer_weights& w = ctx->w[l];
@@ -351,6 +358,9 @@ pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
     r = single_gemm(ctx->om, C, w_last, C, out, C, Mi, C, C, status, s);
     if (r) return r;
   }
+  if (a.layer_events && c.n_layers > 0 &&
+      cudaEventRecord(a.layer_events[c.n_layers], s) != cudaSuccess)
+    return PL_ECUDA;
   r = from_cuda(pl::launch_ddim(ctx->st, ctx->ring, a.eps, a.out_frames, ctx->frame_elems,
                                 ctx->coef, S, s));
   if (r) return r;
@@ -734,6 +744,10 @@ pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_
     delete ctx;
     return PL_ECUDA;
   }
+  {
+    const char* prof = std::getenv("PL_PROFILE");
+    ctx->profile = prof && prof[0] == '1';
+  }
   // zero the device state so pl_get_state is meaningful before bank_init
   if (cudaMemset(ctx->st, 0, sizeof(pl::DevState) * ctx->sessions) != cudaSuccess) {
     delete ctx;
@@ -753,6 +767,8 @@ pl_status pl_ctx_destroy(pl_ctx* ctx) {
     if (ctx->ev_free[b]) cudaEventDestroy(ctx->ev_free[b]);
   }
   if (ctx->copy_stream) cudaStreamDestroy(ctx->copy_stream);
+  for (auto& e : ctx->prof_ev)
+    if (e) cudaEventDestroy(e);
   delete ctx;
   return PL_OK;
 }
@@ -859,8 +875,19 @@ pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_
     if (attn_out && (!attn_out[l] || !aligned16(attn_out[l]))) return PL_EINVAL;
   }
   if (!aligned16(new_noise) || !aligned16(eps) || !aligned16(out_frames)) return PL_EINVAL;
-  RoundArgs a{new_noise, new_motion, hidden, eps, out_frames, appended, layer_out, attn_out};
+  RoundArgs a{new_noise, new_motion, hidden, eps, out_frames, appended, layer_out, attn_out,
+              nullptr};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (ctx->profile) {
+    // profiled rounds run outside the graph, with an event around each layer
+    for (int i = 0; i <= L; ++i)
+      if (!ctx->prof_ev[i] && cudaEventCreate(&ctx->prof_ev[i]) != cudaSuccess) return PL_ECUDA;
+    a.layer_events = ctx->prof_ev;
+    ctx->prof_valid = false;
+    const pl_status r = enqueue_round(ctx, a, s);
+    ctx->prof_valid = r == PL_OK && L > 0;
+    return r;
+  }
   const char* env = std::getenv("PL_NO_GRAPH");
   const bool use_graph = s != nullptr && !(env && env[0] == '1');
   if (!use_graph) return enqueue_round(ctx, a, s);
@@ -913,6 +940,135 @@ pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_
   }
   slot->last_use = ++ctx->graph_tick;
   return from_cuda(cudaGraphLaunch(slot->exec, s));
+}
+
+// ---------------------------------------------------------------- snapshots
+namespace {
+
+constexpr uint64_t kSnapMagic = 0x3130504e53504c50ull;   // "PLSNP01" + version byte
+constexpr uint32_t kSnapVersion = 1;
+
+struct SnapHeader {
+  uint64_t magic;
+  uint32_t version, sessions;
+  int32_t capacity, latent_c, latent_h, latent_w;
+  uint64_t state_bytes, ring_bytes, motion_bytes, bank_bytes;
+};
+
+struct SnapParts {
+  size_t state, ring, motion, bank, total;
+};
+
+SnapParts snap_parts(const pl_ctx* ctx) {
+  SnapParts p;
+  const size_t S = static_cast<size_t>(ctx->sessions);
+  p.state = sizeof(pl::DevState) * S;
+  p.ring = sizeof(float) * S * 16 * static_cast<size_t>(ctx->frame_elems);
+  p.motion = sizeof(float) * S * 16 * 512;
+  p.bank = sizeof(float) * S * static_cast<size_t>(ctx->capacity) * 512;
+  p.total = sizeof(SnapHeader) + p.state + p.ring + p.motion + p.bank;
+  return p;
+}
+
+}  // namespace
+
+pl_status pl_state_bytes(const pl_ctx* ctx, size_t* bytes) {
+  if (!ctx || !bytes) return PL_EINVAL;
+  *bytes = snap_parts(ctx).total;
+  return PL_OK;
+}
+
+pl_status pl_state_export(pl_ctx* ctx, void* host_out, size_t bytes, void* stream) {
+  if (!ctx || !host_out) return PL_EINVAL;
+  if (!ctx->initialised) return PL_ESTATE;
+  const SnapParts sp = snap_parts(ctx);
+  if (bytes < sp.total) return PL_ENOMEM;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PL_ECUDA;
+  SnapHeader h{};
+  h.magic = kSnapMagic;
+  h.version = kSnapVersion;
+  h.sessions = static_cast<uint32_t>(ctx->sessions);
+  h.capacity = ctx->capacity;
+  h.latent_c = ctx->cfg.latent_c;
+  h.latent_h = ctx->cfg.latent_h;
+  h.latent_w = ctx->cfg.latent_w;
+  h.state_bytes = sp.state;
+  h.ring_bytes = sp.ring;
+  h.motion_bytes = sp.motion;
+  h.bank_bytes = sp.bank;
+  uint8_t* o = static_cast<uint8_t*>(host_out);
+  std::memcpy(o, &h, sizeof(h));
+  o += sizeof(h);
+  const struct {
+    const void* src;
+    size_t n;
+  } parts[4] = {{ctx->st, sp.state}, {ctx->ring, sp.ring}, {ctx->slot_motion, sp.motion},
+                {ctx->bank, sp.bank}};
+  for (const auto& pt : parts) {
+    if (cudaMemcpy(o, pt.src, pt.n, cudaMemcpyDeviceToHost) != cudaSuccess) return PL_ECUDA;
+    o += pt.n;
+  }
+  return PL_OK;
+}
+
+pl_status pl_state_import(pl_ctx* ctx, const void* host_in, size_t bytes, void* stream) {
+  if (!ctx || !host_in) return PL_EINVAL;
+  if (!ctx->initialised) return PL_ESTATE;
+  const SnapParts sp = snap_parts(ctx);
+  if (bytes < sp.total) return PL_EINVAL;
+  SnapHeader h;
+  std::memcpy(&h, host_in, sizeof(h));
+  if (h.magic != kSnapMagic || h.version != kSnapVersion ||
+      h.sessions != static_cast<uint32_t>(ctx->sessions) || h.capacity != ctx->capacity ||
+      h.latent_c != ctx->cfg.latent_c || h.latent_h != ctx->cfg.latent_h ||
+      h.latent_w != ctx->cfg.latent_w || h.state_bytes != sp.state || h.ring_bytes != sp.ring ||
+      h.motion_bytes != sp.motion || h.bank_bytes != sp.bank)
+    return PL_EINVAL;
+  const uint8_t* in = static_cast<const uint8_t*>(host_in) + sizeof(h);
+  // the states are checked on the host before anything reaches the device
+  const int S = ctx->sessions;
+  pl::DevState* states = new (std::nothrow) pl::DevState[S];
+  if (!states) return PL_ENOMEM;
+  std::memcpy(states, in, sp.state);
+  for (int z = 0; z < S; ++z) {
+    pl::DevState& d = states[z];
+    bool ok = d.head >= 0 && d.head < 4 && d.bank_count >= 1 && d.bank_count <= ctx->capacity &&
+              d.appends >= 0 && d.appends <= ctx->cfg.append_cap &&
+              d.bank_count == 1 + d.appends && d.rounds >= 0;
+    for (int i = 0; i < 4; ++i) {
+      const int t = d.slot_t[i];
+      ok = ok && (t == -1 || t == 0 || t == 333 || t == 666 || t == 999);
+    }
+    if (!ok) {
+      delete[] states;
+      return PL_EINVAL;
+    }
+    d.status = 0;
+    for (int a = 0; a < 4; ++a) d.anchor_fire[a] = 0;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(ctx->st, states, sp.state, cudaMemcpyHostToDevice);
+  in += sp.state;
+  if (e == cudaSuccess) e = cudaMemcpy(ctx->ring, in, sp.ring, cudaMemcpyHostToDevice);
+  in += sp.ring;
+  if (e == cudaSuccess) e = cudaMemcpy(ctx->slot_motion, in, sp.motion, cudaMemcpyHostToDevice);
+  in += sp.motion;
+  if (e == cudaSuccess) e = cudaMemcpy(ctx->bank, in, sp.bank, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    delete[] states;
+    return PL_ECUDA;
+  }
+  // KV-bank entries 1..appends hold anchors 1..appends projected by each
+  // layer's Wk/Wv: recompute them rather than carry ~185 MB in the snapshot
+  pl_status r = PL_OK;
+  if (ctx->have_anchors) {
+    for (int z = 0; z < S && r == PL_OK; ++z)
+      for (int an = 1; an <= states[z].appends && r == PL_OK; ++an)
+        r = project_bank(ctx, ctx->anchor_feats[an - 1], an, /*predicated=*/false, s, z);
+  }
+  delete[] states;
+  return r;
 }
 
 pl_status pl_host_staging_bytes(const pl_config* cfg, size_t* bytes) {
@@ -1039,6 +1195,24 @@ pl_status pl_get_device_status(pl_ctx* ctx, void* stream) {
   }
   if (w & pl::DEV_TIMEOUT) return PL_ETIMEOUT;
   if (w) return PL_EDEVICE;
+  return PL_OK;
+}
+
+pl_status pl_set_profiling(pl_ctx* ctx, int on) {
+  if (!ctx) return PL_EINVAL;
+  ctx->profile = on != 0;
+  ctx->prof_valid = false;
+  return PL_OK;
+}
+
+pl_status pl_get_layer_ms(pl_ctx* ctx, float* ms_out, int n) {
+  if (!ctx || !ms_out || n < ctx->cfg.n_layers) return PL_EINVAL;
+  if (!ctx->prof_valid) return PL_ESTATE;
+  const int L = ctx->cfg.n_layers;
+  if (cudaEventSynchronize(ctx->prof_ev[L]) != cudaSuccess) return PL_ECUDA;
+  for (int l = 0; l < L; ++l)
+    if (cudaEventElapsedTime(&ms_out[l], ctx->prof_ev[l], ctx->prof_ev[l + 1]) != cudaSuccess)
+      return PL_ECUDA;
   return PL_OK;
 }
 

@@ -565,6 +565,38 @@ pl_status pl_get_session_motion_bank(pl_ctx* ctx, int session, float* host_out, 
  * status: PL_OK, PL_ETIMEOUT or PL_EDEVICE. Clears the words. */
 pl_status pl_get_device_status(pl_ctx* ctx, void* stream);
 
+/* Per-layer timing (no counterpart in the pages). With profiling on (this
+ * call, or PL_PROFILE=1 in the environment when the context is created),
+ * pl_stream_round runs the round outside its captured graph with a CUDA
+ * event before each layer and after the last; pl_get_layer_ms synchronises
+ * on the last event and writes the n_layers layer times (reference attention
+ * plus motion cross-attention, ms) of the latest profiled round to ms_out
+ * (host, n >= n_layers), or returns PL_ESTATE when there is none. The
+ * events cost a few microseconds per layer; the graph path is unaffected
+ * when profiling is off. */
+pl_status pl_set_profiling(pl_ctx* ctx, int on);
+pl_status pl_get_layer_ms(pl_ctx* ctx, float* ms_out, int n);
+
+/* Checkpoint and resume of the streams' state (no counterpart in the pages,
+ * which pause and reset a stream but do not resume one; the state is small
+ * and device-resident, so it is the natural unit to save).
+ * pl_state_bytes: host bytes of a snapshot: a header, then per session the
+ * device state (pile head, slot timesteps, bank count, appends, counters),
+ * the pile's latents [16][latent_c][H][W] fp32, the slots' motion
+ * embeddings [16][512] and the motion bank [capacity][512].
+ * pl_state_export: synchronise `stream` and copy the snapshot to host_out
+ * (host memory of >= pl_state_bytes; PL_ESTATE before pl_bank_init).
+ * pl_state_import: restore a snapshot into a context of the same
+ * configuration after its pl_bank_init (weights, reference and anchor
+ * features given again): the header and every state are checked on the host
+ * (PL_EINVAL on any mismatch, nothing written then); the KV-bank rows of the
+ * appended anchors are projected again from the anchor features instead of
+ * being stored. Rounds after an import continue the exported stream: same
+ * inputs give the same outputs, bit for bit. Both calls block. */
+pl_status pl_state_bytes(const pl_ctx* ctx, size_t* bytes);
+pl_status pl_state_export(pl_ctx* ctx, void* host_out, size_t bytes, void* stream);
+pl_status pl_state_import(pl_ctx* ctx, const void* host_in, size_t bytes, void* stream);
+
 /* Synchronise `stream`, then read and clear the current device's status word
  * of context-free calls (see the conventions above): PL_OK, PL_ETIMEOUT (a
  * bounded wait gave up) or PL_EDEVICE (a kernel refused its arguments). The

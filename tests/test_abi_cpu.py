@@ -140,6 +140,17 @@ def test_host_staging_size_and_validation():
                                       None) == P.PL_EINVAL
 
 
+def test_state_and_profiling_calls_validate_their_arguments():
+    import denoise_step_b200 as P
+    n = C.c_size_t()
+    assert P.lib.pl_state_bytes(None, C.byref(n)) == P.PL_EINVAL
+    assert P.lib.pl_state_export(None, None, 0, None) == P.PL_EINVAL
+    assert P.lib.pl_state_import(None, None, 0, None) == P.PL_EINVAL
+    assert P.lib.pl_set_profiling(None, 1) == P.PL_EINVAL
+    buf = (C.c_float * 4)()
+    assert P.lib.pl_get_layer_ms(None, buf, 4) == P.PL_EINVAL
+
+
 def test_round_before_init_is_a_state_error():
     import denoise_step_b200 as P
     # a null context is rejected before any device work
