@@ -140,6 +140,24 @@ def test_host_staging_size_and_validation():
                                       None) == P.PL_EINVAL
 
 
+def test_large_bank_check_needs_its_workspace():
+    import denoise_step_b200 as P
+    L = P.lib
+    fake = C.c_void_p(1 << 20)                 # never dereferenced: rejected on the host
+    n = C.c_size_t()
+    assert L.pl_motion_bank_check_workspace_bytes(100000, 512, 4, C.byref(n)) == P.PL_OK
+    need = n.value
+    args = (fake, fake, fake, 100000, 512, fake, 4, 17.0, 3, None, None, None)
+    assert L.pl_motion_bank_check(*args, None, 0, None) == P.PL_EINVAL          # no workspace
+    assert L.pl_motion_bank_check(*args, fake, need - 1, None) == P.PL_ENOMEM  # too small
+    assert L.pl_motion_bank_check(*args, C.c_void_p((1 << 20) + 8), need,
+                                  None) == P.PL_EINVAL                          # misaligned
+    # queries x dim past the shared-memory budget of the multi-CTA pass
+    assert L.pl_motion_bank_check_workspace_bytes(100000, 4096, 8, C.byref(n)) == P.PL_OK
+    assert L.pl_motion_bank_check(fake, fake, fake, 100000, 4096, fake, 8, 17.0, 3, None, None,
+                                  None, fake, n.value, None) == P.PL_EUNSUPPORTED
+
+
 def test_state_and_profiling_calls_validate_their_arguments():
     import denoise_step_b200 as P
     n = C.c_size_t()
