@@ -18,7 +18,7 @@ Sources (web pages; cited by page and section):
 Every function computes the plain definition in float64 with library matmuls
 as the only primitive; nothing is blocked, fused or reordered.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent (the plainest reading the rest supports):
   * beta schedule: SD "scaled linear", beta_start 0.00085, beta_end 0.012,
     1000 steps (the pages name DDIM with epsilon prediction and the SD VAE
     scale 0.18215 but print no schedule);
@@ -410,7 +410,7 @@ def prefill_motion(ref_motion, drive0_motion, frames: int = 12) -> np.ndarray:
 # keypoints with pitch / yaw / roll / translation / scale; retargeting keeps
 # the reference's canonical keypoints and scale, takes only the driving
 # rotation and half its translation; 7 of the 21 points are drawn as coloured
-# dots. Readings where the page is silent (listed in the design doc): angles in
+# dots. Readings where the page is silent (the plainest consistent one): angles in
 # degrees, R = Rz(roll) Ry(yaw) Rx(pitch) acting on column vectors; keypoint
 # = scale * R c + 0.5 t; the dot image is orthographic with x, y in [-1, 1]
 # mapped to [0, W] x [0, H] (z dropped); a pixel (centre (x + 0.5, y + 0.5))
