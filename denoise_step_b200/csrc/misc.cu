@@ -1,5 +1,7 @@
 #include <cmath>
 
+#include "devinit.cuh"
+#include "fastmath.cuh"
 #include "misc.cuh"
 #include "ptx.cuh"
 
@@ -368,8 +370,11 @@ constexpr int kBankMaxQueries = 64;
 
 __global__ void __launch_bounds__(kBankThreads) bank_partial_kernel(
     const float* __restrict__ bank, const int32_t* count_p, int64_t capacity, int dim,
-    const float* __restrict__ queries, int nq, double* part_d2, int64_t* part_idx) {
+    const float* __restrict__ queries, int nq, double* part_d2, int64_t* part_idx,
+    const int32_t* need) {
   extern __shared__ double sq[];                    // [nq][dim]
+  // run only when the fp32 screen left a query undecided
+  if (need != nullptr && *((volatile const int32_t*)need) == 0) return;
   __shared__ double w_best[kBankThreads / 32][kBankMaxQueries];
   __shared__ int64_t w_idx[kBankThreads / 32][kBankMaxQueries];
   constexpr int kSlots = 32 / kBankLanes;
@@ -505,12 +510,230 @@ __global__ void __launch_bounds__(kBankThreads) bank_partial_kernel(
   }
 }
 
+// Large banks, fp32 screen: the traversal of the fp64 pass (four lanes per
+// entry, each walking its quarter of the row in 16-byte chunks; queries in
+// shared memory) with fp32 arithmetic, which needs half the registers: three
+// CTAs per SM instead of two, so more rows in flight (the fp64 pass and this
+// one are bound by the loads in flight, not by their arithmetic: at 262144 x
+// 512 with 4 queries, fp32 with two CTAs per SM ran as fast as fp64, a warp per
+// row with the queries in registers (one CTA per SM) 45% slower, and eight
+// entries per lane (one CTA per SM) 10% slower). Per query it keeps the smallest
+// computed d^2 (its index, lowest on ties) and the second smallest. Rounding
+// bound: each lane sums its n = dim / 4 terms (q - x)^2 with one fma per term,
+// the subtraction rounded once, and two shuffle additions join the lanes, so
+// the computed value is within (n + 4) u of the exact d^2, relative (u =
+// 2^-24, all terms non-negative): 132 u ~ 7.9e-6 at dim 512. When the second
+// smallest exceeds the smallest by more than twice that bound, the smallest
+// is the exact argmin and the fp64 pass is not needed; bank_select_kernel
+// asks for a gap of 4e-5 (a 2.5x margin at dim 512), scaled with n past it.
+__device__ __forceinline__ void top2_push(float c, int64_t j, float& b1, int64_t& i1, float& b2) {
+  if (c < b1) {
+    b2 = b1;
+    b1 = c;
+    i1 = j;
+  } else if (c < b2) {
+    b2 = c;
+  }
+}
+// merge (o1, oi, o2) into (b1, i1, b2): lowest index first on equal values;
+// the same entry seen twice (the lanes that share an entry all hold its sum)
+// counts once
+__device__ __forceinline__ void top2_merge(float& b1, int64_t& i1, float& b2, float o1, int64_t oi,
+                                           float o2) {
+  if (oi < 0) return;
+  if (oi == i1) {
+    b2 = fminf(b2, o2);
+    return;
+  }
+  if (i1 < 0 || o1 < b1 || (o1 == b1 && oi < i1)) {
+    b2 = fminf(b1, o2);
+    b1 = o1;
+    i1 = oi;
+  } else {
+    b2 = fminf(b2, o1);
+  }
+}
+
+constexpr int kScreenE = 4;        // entries per lane at once
+constexpr int kScreenBlocks = 3;   // CTAs per SM (80 registers a thread)
+
+__global__ void __launch_bounds__(kBankThreads, kScreenBlocks) bank_screen_kernel(
+    const float* __restrict__ bank, const int32_t* count_p, int64_t capacity, int dim,
+    const float* __restrict__ queries, int nq, float* part_b1, int64_t* part_i1, float* part_b2) {
+  extern __shared__ float sqf[];                    // [nq][dim]
+  __shared__ float w_b1[kBankThreads / 32][kBankMaxQueries];
+  __shared__ float w_b2[kBankThreads / 32][kBankMaxQueries];
+  __shared__ int64_t w_i1[kBankThreads / 32][kBankMaxQueries];
+  constexpr int kSlots = 32 / kBankLanes;
+  constexpr int kPerWarp = kSlots * kScreenE;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane % kBankLanes, slot = lane / kBankLanes;
+  for (int i = threadIdx.x; i < nq * dim; i += kBankThreads) sqf[i] = queries[i];
+  __syncthreads();
+  int64_t cnt = *count_p;
+  cnt = cnt < 0 ? 0 : (cnt > capacity ? capacity : cnt);
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * (kBankThreads / 32) + warp;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (kBankThreads / 32);
+  for (int g0 = 0; g0 < nq; g0 += kBankGroup) {
+    const int gn = nq - g0 < kBankGroup ? nq - g0 : kBankGroup;
+    const float* q0 = sqf + static_cast<int64_t>(g0) * dim;
+    float b1[kBankGroup], b2[kBankGroup];
+    int64_t i1[kBankGroup];
+#pragma unroll
+    for (int g = 0; g < kBankGroup; ++g) {
+      b1[g] = INFINITY;
+      b2[g] = INFINITY;
+      i1[g] = -1;
+    }
+    for (int64_t j0 = gw * kPerWarp; j0 < cnt; j0 += nw * kPerWarp) {
+      // a lane's entries: j0 + slot + kSlots * u, increasing
+      float acc[kScreenE][kBankGroup];
+#pragma unroll
+      for (int u = 0; u < kScreenE; ++u)
+#pragma unroll
+        for (int g = 0; g < kBankGroup; ++g) acc[u][g] = 0.f;
+      const float* e[kScreenE];
+      bool ok[kScreenE];
+#pragma unroll
+      for (int u = 0; u < kScreenE; ++u) {
+        const int64_t j = j0 + slot + kSlots * u;
+        ok[u] = j < cnt;
+        e[u] = bank + (ok[u] ? j : 0) * dim;   // rows past the end read row 0, unused
+      }
+      for (int d = 4 * sub; d < dim; d += 4 * kBankLanes) {
+        float4 x[kScreenE];
+#pragma unroll
+        for (int u = 0; u < kScreenE; ++u) x[u] = __ldg(reinterpret_cast<const float4*>(e[u] + d));
+#pragma unroll
+        for (int g = 0; g < kBankGroup; ++g) {
+          if (g < gn) {
+            const float4 q = *reinterpret_cast<const float4*>(q0 + g * dim + d);
+#pragma unroll
+            for (int u = 0; u < kScreenE; ++u) {
+              const float d0 = q.x - x[u].x, d1 = q.y - x[u].y;
+              const float d2 = q.z - x[u].z, d3 = q.w - x[u].w;
+              acc[u][g] = fmaf(d3, d3, fmaf(d2, d2, fmaf(d1, d1, fmaf(d0, d0, acc[u][g]))));
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kScreenE; ++u) {
+#pragma unroll
+        for (int g = 0; g < kBankGroup; ++g) {
+          if (g < gn) {
+#pragma unroll
+            for (int o = 1; o < kBankLanes; o <<= 1)
+              acc[u][g] += __shfl_xor_sync(0xffffffffu, acc[u][g], o);
+            if (ok[u]) top2_push(acc[u][g], j0 + slot + kSlots * u, b1[g], i1[g], b2[g]);
+          }
+        }
+      }
+    }
+    // warp state per query: the lanes of an entry hold the same candidates,
+    // which the merge counts once
+#pragma unroll
+    for (int g = 0; g < kBankGroup; ++g) {
+      if (g < gn) {
+        float a1 = b1[g], a2 = b2[g];
+        int64_t ai = i1[g];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float o1 = __shfl_xor_sync(0xffffffffu, a1, o);
+          const float o2 = __shfl_xor_sync(0xffffffffu, a2, o);
+          const int64_t oi = __shfl_xor_sync(0xffffffffu, ai, o);
+          top2_merge(a1, ai, a2, o1, oi, o2);
+        }
+        if (lane == 0) {
+          w_b1[warp][g0 + g] = a1;
+          w_b2[warp][g0 + g] = a2;
+          w_i1[warp][g0 + g] = ai;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < nq; k += kBankThreads) {
+    float a1 = INFINITY, a2 = INFINITY;
+    int64_t ai = -1;
+    for (int w = 0; w < kBankThreads / 32; ++w) top2_merge(a1, ai, a2, w_b1[w][k], w_i1[w][k], w_b2[w][k]);
+    const int64_t o = static_cast<int64_t>(blockIdx.x) * nq + k;
+    part_b1[o] = a1;
+    part_b2[o] = a2;
+    part_i1[o] = ai;
+  }
+}
+
+// the screen's layout: rows of a multiple of 4 floats, 16-byte aligned
+bool bank_screen_ok(int dim, const float* bank, const float* queries) {
+  return dim % 4 == 0 &&
+         ((reinterpret_cast<uintptr_t>(bank) | reinterpret_cast<uintptr_t>(queries)) & 15) == 0;
+}
+
+constexpr float kBankScreenGap = 4e-5f;
+
+// Large banks, screen decision (one CTA): per query the screen's nearest entry
+// and whether it is certain; need = 1 when any query needs the fp64 pass.
+__global__ void set_flag_kernel(int32_t* flag, int32_t v) { *flag = v; }
+
+__global__ void __launch_bounds__(kBankThreads) bank_select_kernel(
+    const int32_t* count_p, int64_t capacity, int dim, int nq, const float* part_b1,
+    const int64_t* part_i1, const float* part_b2, int parts, int64_t* sel_idx, int32_t* need) {
+  __shared__ int s_need;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) s_need = 0;
+  __syncthreads();
+  int64_t cnt = *count_p;
+  cnt = cnt < 0 ? 0 : (cnt > capacity ? capacity : cnt);
+  // twice the rounding bound (n + 4) u with a 2.5x margin, n = dim / 4
+  const float gap = kBankScreenGap * fmaxf(1.0f, (dim / kBankLanes + 4) / 132.0f);
+  for (int k = warp; k < nq; k += kBankThreads / 32) {
+    float a1 = INFINITY, a2 = INFINITY;
+    int64_t ai = -1;
+    // eight partials per lane loaded before any is merged (one load latency
+    // per batch, not per partial)
+    for (int p0 = 0; p0 < parts; p0 += 8 * 32) {
+      float l1[8], l2[8];
+      int64_t li[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int pt = p0 + r * 32 + lane;
+        const int64_t o = static_cast<int64_t>(pt < parts ? pt : 0) * nq + k;
+        l1[r] = part_b1[o];
+        l2[r] = part_b2[o];
+        li[r] = pt < parts ? part_i1[o] : -1;
+      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r) top2_merge(a1, ai, a2, l1[r], li[r], l2[r]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float o1 = __shfl_xor_sync(0xffffffffu, a1, o);
+      const float o2 = __shfl_xor_sync(0xffffffffu, a2, o);
+      const int64_t oi = __shfl_xor_sync(0xffffffffu, ai, o);
+      top2_merge(a1, ai, a2, o1, oi, o2);
+    }
+    if (lane == 0) {
+      // certain: no entry; or a candidate that is the only entry or leads
+      // the runner-up by a finite gap past the rounding bound (an overflow to
+      // infinity, a NaN or a near-zero pair leaves the query to the fp64 pass)
+      const bool certain =
+          cnt == 0 || (ai >= 0 && (cnt == 1 || (a2 < INFINITY && a2 > 1e-20f && a2 - a1 > gap * a2)));
+      sel_idx[k] = cnt == 0 ? -1 : ai;
+      if (!certain) atomicOr(&s_need, 1);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) *need = s_need;
+}
+
 // Large banks, pass 2 (one CTA): per query the minimum over the partial
 // minima, the query-query distances, the in-order decisions and the copies.
 __global__ void __launch_bounds__(kBankThreads) bank_resolve_kernel(
     float* bank, int32_t* count_p, int32_t* appends_p, int capacity, int dim,
     const float* __restrict__ queries, int nq, double thr2, int cap, const double* part_d2,
-    const int64_t* part_idx, int parts, int32_t* argmin, double* min_d2, uint8_t* appended) {
+    const int64_t* part_idx, int parts, const int64_t* sel_idx, const int32_t* need,
+    int32_t* argmin, double* min_d2, uint8_t* appended) {
   __shared__ double s_dq[kBankMaxQueries * kBankMaxQueries];
   __shared__ double s_bd[kBankMaxQueries];
   __shared__ int s_bi[kBankMaxQueries], s_list[kBankMaxQueries];
@@ -522,8 +745,22 @@ __global__ void __launch_bounds__(kBankThreads) bank_resolve_kernel(
     s_cnt0 = c < 0 ? 0 : (c > capacity ? capacity : c);
     s_app0 = *appends_p;
   }
+  const bool screened = need != nullptr && *((volatile const int32_t*)need) == 0;
+  if (screened) {
+    // the screen fixed every nearest stored entry: its exact fp64 d^2
+    for (int k = warp; k < nq; k += nwarps) {
+      const int64_t j = sel_idx[k];
+      const double d = j >= 0 ? dist2_warp(queries + static_cast<int64_t>(k) * dim,
+                                           bank + j * static_cast<int64_t>(dim), dim, lane)
+                              : INFINITY;
+      if (lane == 0) {
+        s_bd[k] = d;
+        s_bi[k] = static_cast<int>(j);
+      }
+    }
+  }
   // per query: one warp reduces the partial minima (lowest index on ties)
-  for (int k = warp; k < nq; k += nwarps) {
+  for (int k = warp; !screened && k < nq; k += nwarps) {
     double b = INFINITY;
     int64_t bi = -1;
     for (int pt = lane; pt < parts; pt += 32) {
@@ -980,9 +1217,14 @@ int bank_parts(int64_t capacity) {
 
 bool bank_small(int capacity, int nq) { return capacity <= kBankSmall && nq <= kBankSmall; }
 
+// large-path workspace: fp64 partials (d2, index), the screen's partials
+// (index, best, second best), the screen's picks and, in the int32 at 16
+// bytes before the end, the fp64-pass flag of the last call (1 = it ran)
 size_t bank_workspace_bytes(int64_t capacity, int nq) {
   if (bank_small(static_cast<int>(capacity > 1 << 30 ? 1 << 30 : capacity), nq)) return 0;
-  return static_cast<size_t>(bank_parts(capacity)) * nq * (sizeof(double) + sizeof(int64_t));
+  const size_t pn = static_cast<size_t>(bank_parts(capacity)) * nq;
+  return pn * (sizeof(double) + 2 * sizeof(int64_t) + 2 * sizeof(float)) +
+         static_cast<size_t>(nq) * sizeof(int64_t) + 16;
 }
 
 cudaError_t launch_bank_check(float* bank, int32_t* count, int32_t* appends, int capacity,
@@ -1000,18 +1242,49 @@ cudaError_t launch_bank_check(float* bank, int32_t* count, int32_t* appends, int
   // large banks: context-free calls only (one session, caller workspace)
   if (st || !workspace) return cudaErrorInvalidValue;
   const size_t smem = sizeof(double) * static_cast<size_t>(nq) * dim;
+  const size_t smem32 = smem / 2;
   if (smem > 160 * 1024) return cudaErrorInvalidValue;
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(bank_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return cudaErrorInvalidValue;
+  if (smem32 > 48 * 1024 &&
+      cudaFuncSetAttribute(bank_screen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem32)) != cudaSuccess)
+    return cudaErrorInvalidValue;
   const int parts = bank_parts(capacity);
+  const size_t pn = static_cast<size_t>(parts) * nq;
   double* pd = static_cast<double*>(workspace);
-  int64_t* pi = reinterpret_cast<int64_t*>(pd + static_cast<size_t>(parts) * nq);
-  bank_partial_kernel<<<parts, kBankThreads, smem, s>>>(bank, count, capacity, dim, queries, nq, pd,
-                                                        pi);
+  int64_t* pi = reinterpret_cast<int64_t*>(pd + pn);
+  int64_t* si1 = pi + pn;
+  int64_t* sel = si1 + pn;
+  float* sb1 = reinterpret_cast<float*>(sel + nq);
+  float* sb2 = sb1 + pn;
+  int32_t* need = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
+                                             bank_workspace_bytes(capacity, nq) - 16);
+  // fp32 screen, its decision, the fp64 pass only when a query is undecided,
+  // then the in-order decisions (rows the screen does not take: the fp64
+  // pass decides alone)
+  const bool screen = bank_screen_ok(dim, bank, queries);
+  // both passes stride over the entries: persistent grids of as many CTAs as
+  // fit on the SMs (fewer partials to merge, a cheap exit for the fp64 pass
+  // when it is not needed)
+  const int sms = device_sms();
+  const int fparts = sms > 0 && parts > 2 * sms ? 2 * sms : parts;
+  if (screen) {
+    const int sparts = sms > 0 && parts > sms * kScreenBlocks ? sms * kScreenBlocks : parts;
+    bank_screen_kernel<<<sparts, kBankThreads, smem32, s>>>(bank, count, capacity, dim, queries, nq,
+                                                            sb1, si1, sb2);
+    bank_select_kernel<<<1, kBankThreads, 0, s>>>(count, capacity, dim, nq, sb1, si1, sb2, sparts,
+                                                  sel, need);
+  } else {
+    set_flag_kernel<<<1, 1, 0, s>>>(need, 1);
+  }
+  bank_partial_kernel<<<fparts, kBankThreads, smem, s>>>(bank, count, capacity, dim, queries, nq,
+                                                         pd, pi, need);
   bank_resolve_kernel<<<1, kBankThreads, 0, s>>>(bank, count, appends, capacity, dim, queries, nq,
-                                                 thr2, cap, pd, pi, parts, argmin, min_d2, appended);
+                                                 thr2, cap, pd, pi, fparts, sel, need, argmin,
+                                                 min_d2, appended);
   return cudaGetLastError();
 }
 cudaError_t launch_nearest(const float* store, int count, int dim, const float* query,

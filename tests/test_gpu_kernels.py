@@ -177,7 +177,10 @@ def test_motion_xattn(P, N, C):
 
 # ------------------------------------------------------------------ motion bank
 
-def _bank_run(P, bank_np, count, queries, thr, cap, capacity):
+def _bank_run(P, bank_np, count, queries, thr, cap, capacity, flag=None):
+    """One bank check on the device. `flag` (a list) receives, for the large
+    path, whether the fp64 pass ran: the int32 16 bytes before the end of the
+    workspace (0 = the fp32 screen settled every nearest entry)."""
     dim = bank_np.shape[1]
     bank = torch.zeros((capacity, dim), dtype=torch.float32, device="cuda")
     bank[:count] = dev(bank_np[:count])
@@ -187,8 +190,14 @@ def _bank_run(P, bank_np, count, queries, thr, cap, capacity):
     am = torch.full((nq,), -7, dtype=torch.int32, device="cuda")
     d2 = torch.zeros(nq, dtype=torch.float64, device="cuda")
     fl = torch.zeros(nq, dtype=torch.uint8, device="cuda")
-    P.motion_bank_check(bank, cnt, app, dev(np.asarray(queries, np.float32)), thr, cap, am, d2, fl)
+    need = P.sz()
+    P.check(P.lib.pl_motion_bank_check_workspace_bytes(capacity, dim, nq, P.C.byref(need)), "ws")
+    ws = torch.full((max(need.value, 16),), 0x55, dtype=torch.uint8, device="cuda")
+    P.motion_bank_check(bank, cnt, app, dev(np.asarray(queries, np.float32)), thr, cap, am, d2, fl,
+                        workspace=ws if need.value > 0 else None)
     torch.cuda.synchronize()
+    if flag is not None and need.value > 0:
+        flag.append(int(ws[need.value - 16:need.value - 12].view(torch.int32).item()))
     return host(bank), int(cnt.item()), int(app.item()), host(am), host(d2), host(fl)
 
 
@@ -240,12 +249,57 @@ def test_bank_check_large_banks_bit_exact(P, count, dim, nq):
             qs[k] = bank[pick[k]] + jit[k]
         elif k % 3 == 2 and k >= 2:
             qs[k] = qs[k - 2] + jit[k]
-    gbank, cnt, app, am, d2, fl = _bank_run(P, bank, count, qs, 17.0, 3, count + 3)
+    flag = []
+    gbank, cnt, app, am, d2, fl = _bank_run(P, bank, count, qs, 17.0, 3, count + 3, flag)
     w_am, w_d2, w_fl, w_bank, w_app = O.bank_check(list(bank), list(qs), 0)
     assert list(am) == w_am and list(fl) == w_fl and app == w_app and cnt == len(w_bank)
     assert np.max(np.abs(d2 - np.array(w_d2)) / np.maximum(np.array(w_d2), 1e-300)) < 1e-12
     assert np.array_equal(gbank[:cnt], np.array(w_bank, np.float32))
     assert w_fl[0] == 1 and w_am[2] == count        # query 2 finds query 0's appended copy
+    # no near-tie among these: the fp32 screen decides alone where it takes the
+    # rows (multiples of 4 floats up to 512), else the fp64 pass runs
+    assert flag == [0 if dim % 4 == 0 and dim <= 512 else 1]
+
+
+def test_bank_check_large_bank_ties_take_the_fp64_pass(P):
+    # Exact duplicates among the stored entries tie in every precision, so the
+    # fp32 screen cannot settle those queries' nearest entry and the fp64 pass
+    # decides (lowest index on ties): query 0 sits next to entry 1234 (copied
+    # to 3000), query 1 next to entry 77 (copied to 78 and 4000), query 2 is
+    # far from everything (appended).
+    seed = 73
+    count, dim = 5000, 64
+    bank = S.normal(seed, "tb", (count, dim), 2.0, np.float32)
+    bank[3000] = bank[1234]
+    bank[78] = bank[77]
+    bank[4000] = bank[77]
+    jit = S.normal(seed, "tj", (2, dim), 0.05, np.float32)
+    far = S.normal(seed, "tf", (1, dim), 6.0, np.float32)
+    qs = np.stack([bank[1234] + jit[0], bank[77] + jit[1], far[0]]).astype(np.float32)
+    flag = []
+    gbank, cnt, app, am, d2, fl = _bank_run(P, bank, count, qs, 17.0, 3, count + 3, flag)
+    assert flag == [1]
+    w_am, w_d2, w_fl, w_bank, w_app = O.bank_check(list(bank), list(qs), 0)
+    assert w_am[:2] == [1234, 77] and w_fl == [0, 0, 1]
+    assert list(am) == w_am and list(fl) == w_fl and app == w_app and cnt == len(w_bank)
+    assert np.max(np.abs(d2 - np.array(w_d2)) / np.array(w_d2)) < 1e-12
+    assert np.array_equal(gbank[:cnt], np.array(w_bank, np.float32))
+
+
+def test_bank_check_large_path_single_entry(P):
+    # a capacity past the one-CTA path with one stored entry: the screen has no
+    # runner-up, its pick stands; every query is far, so the first three are
+    # appended and later ones find those copies
+    seed = 74
+    bank = S.normal(seed, "sb", (1, 128), 2.0, np.float32)
+    qs = S.normal(seed, "sq", (5, 128), 2.0, np.float32)
+    flag = []
+    gbank, cnt, app, am, d2, fl = _bank_run(P, bank, 1, qs, 17.0, 3, 40, flag)
+    assert flag == [0]
+    w_am, w_d2, w_fl, w_bank, w_app = O.bank_check(list(bank), list(qs), 0)
+    assert list(am) == w_am and list(fl) == w_fl and app == w_app and cnt == len(w_bank)
+    assert np.max(np.abs(d2 - np.array(w_d2)) / np.array(w_d2)) < 1e-12
+    assert np.array_equal(gbank[:cnt], np.array(w_bank, np.float32))
 
 
 def test_pose_retrieval_argmin(P):
