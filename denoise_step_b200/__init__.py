@@ -118,6 +118,7 @@ _SIGS = {
     "pl_get_device_status": (i32, [vp, vp]),
     "pl_set_profiling": (i32, [vp, i32]),
     "pl_get_layer_ms": (i32, [vp, vp, i32]),
+    "pl_round_kernel_count": (i32, [vp, vp]),
     "pl_state_bytes": (i32, [vp, C.POINTER(sz)]),
     "pl_state_export": (i32, [vp, vp, sz, vp]),
     "pl_state_import": (i32, [vp, vp, sz, vp]),
@@ -498,6 +499,12 @@ class Stream:
         buf = (C.c_float * max(L, 1))()
         check(lib.pl_get_layer_ms(self.handle, buf, L), "pl_get_layer_ms")
         return [buf[i] for i in range(L)]
+
+    def round_kernels(self) -> int:
+        """Kernels one round launches, counted in the captured round graph."""
+        n = i32()
+        check(lib.pl_round_kernel_count(self.handle, C.byref(n)), "pl_round_kernel_count")
+        return n.value
 
     def export_state(self, stream=None):
         """Snapshot of the streams' state as a numpy uint8 array (blocks)."""

@@ -211,6 +211,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_f16_kernel(const __grid_cons
         }
         const int x = tc.n0 + c0;
         if (!rows_in || x >= pr.N) continue;
+        if (pr.softmax32) {
+          // the chunk is one 32-column group (tiles start at multiples of 32):
+          // p = 2^(v - max) / sum over the group, per row
+          float m = __uint_as_float(r[0]);
+#pragma unroll
+          for (int j = 1; j < 32; ++j) m = fmaxf(m, __uint_as_float(r[j]));
+          float sum = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float e = exp2f(__uint_as_float(r[j]) - m);
+            sum += e;
+            r[j] = __float_as_uint(e);
+          }
+          const float inv = 1.0f / sum;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * inv);
+        }
         // the slot's previous store must have finished reading it
         if (lane == 0) bulk_wait_read<1>();
         __syncwarp();
@@ -286,11 +303,19 @@ int gemm_make_problem(GemmProblem* p, const void* a, int64_t lda, const void* b,
     if (encode_tmap(&p->c, out_f32, c, 2, dims, strides, box, out_f32 ? 128 : 64) != 0) return 2;
   }
   p->out_f32 = out_f32 ? 1 : 0;
+  p->softmax32 = 0;
   p->M = M;
   p->N = N;
   p->K = K;
   p->tiles_n = (N + kGemmBN - 1) / kGemmBN;
   p->pred = pred;
+  return 0;
+}
+
+int gemm_set_softmax32(GemmProblem* p) {
+  static_assert(kGemmBN % 32 == 0, "tiles start on 32-column groups");
+  if (p->out_f32 || p->N % 32) return 1;
+  p->softmax32 = 1;
   return 0;
 }
 

@@ -21,6 +21,8 @@ struct GemmProblem {
   CUtensorMap c;        // 2D {N, M}, box {32, 32}: fp16 with 64-byte swizzle or
                         // fp32 (out_f32) with 128-byte swizzle; stored by TMA
   int out_f32;
+  int softmax32;              // fp16 output, each 32-column group replaced by the
+                              // softmax of its values taken as base-2 logits
   int M, N, K;
   int tiles_n;
   int tile_begin, tile_end;   // linear tile range [begin, end)
@@ -40,6 +42,9 @@ int gemm_make_problem(GemmProblem* p, const void* a, int64_t lda, const void* b,
                       bool out_f32 = false);
 // Set kernel attributes once (call outside stream capture). 0 on success.
 int gemm_init();
+// Turn a problem's epilogue into the 32-column softmax (fp16 output, N a
+// multiple of 32). 0 on success.
+int gemm_set_softmax32(GemmProblem* p);
 // Launch a grouped GEMM over params->prob[0..n_problems). Fills tile ranges.
 int gemm_launch(GemmParams* params, cudaStream_t stream, int max_ctas);
 

@@ -1322,6 +1322,72 @@ cudaError_t launch_motion_kv(const float* motion, const __half* m_kv, int F, int
   return cudaGetLastError();
 }
 
+// Motion cross-attention folded for frame f and head h (32 tokens t, head
+// channels d < hd = C / H): with the block's query projection Wq and output
+// projection Mo,
+//   W_qk[f][c][32 h + t] = fp16(alpha * sum_d Wq[c][hd h + d] K[f][t][hd h + d])
+//   VM[f][32 h + t][c]   = fp16(sum_d V[f][t][hd h + d] Mo[hd h + d][c])
+// so the block's scores for input rows X are X W_qk[f] (alpha = log2 e /
+// sqrt(hd): base-2 logits) and its output is sum_h P_h VM_h = (P V) Mo. Sums
+// in fp32, one rounding. Block (h, f, z): rows c of W_qk and columns c of VM
+// from 256 z on.
+__global__ void __launch_bounds__(256) motion_fold_kernel(const float* __restrict__ kv,
+                                                          const __half* __restrict__ wq,
+                                                          const __half* __restrict__ mo, int C,
+                                                          int H, float alpha, __half* wqk,
+                                                          __half* vm) {
+  extern __shared__ float skv[];   // K then V of the head: [2][32][hd]
+  const int h = blockIdx.x, f = blockIdx.y;
+  const int hd = C / H, NT = 32 * H;
+  const float* base = kv + static_cast<int64_t>(f) * 32 * 2 * C;
+  for (int i = threadIdx.x; i < 32 * hd; i += blockDim.x) {
+    const int t = i / hd, d = i - t * hd;
+    skv[i] = base[static_cast<int64_t>(t) * 2 * C + h * hd + d];
+    skv[32 * hd + i] = base[static_cast<int64_t>(t) * 2 * C + C + h * hd + d];
+  }
+  __syncthreads();
+  const float* sk = skv;
+  const float* sv = skv + 32 * hd;
+  const int c = blockIdx.z * blockDim.x + threadIdx.x;
+  if (c >= C) return;
+  float acc[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) acc[t] = 0.f;
+  const __half* wrow = wq + static_cast<int64_t>(c) * C + h * hd;
+  for (int d = 0; d < hd; ++d) {
+    const float w = __half2float(wrow[d]);
+#pragma unroll
+    for (int t = 0; t < 32; ++t) acc[t] = fmaf(w, sk[t * hd + d], acc[t]);
+  }
+  __half* o = wqk + (static_cast<int64_t>(f) * C + c) * NT + 32 * h;
+#pragma unroll
+  for (int t = 0; t < 32; t += 2)
+    *reinterpret_cast<__half2*>(o + t) = __floats2half2_rn(alpha * acc[t], alpha * acc[t + 1]);
+#pragma unroll
+  for (int t = 0; t < 32; ++t) acc[t] = 0.f;
+  for (int d = 0; d < hd; ++d) {
+    const float m = __half2float(mo[static_cast<int64_t>(h * hd + d) * C + c]);
+#pragma unroll
+    for (int t = 0; t < 32; ++t) acc[t] = fmaf(sv[t * hd + d], m, acc[t]);
+  }
+  __half* v = vm + (static_cast<int64_t>(f) * NT + 32 * h) * C + c;
+#pragma unroll
+  for (int t = 0; t < 32; ++t) v[static_cast<int64_t>(t) * C] = __float2half_rn(acc[t]);
+}
+
+cudaError_t launch_motion_fold(const float* kv, const __half* wq, const __half* mo, int F, int C,
+                               int heads, __half* wqk, __half* vm, cudaStream_t s) {
+  if (heads < 1 || C % heads) return cudaErrorInvalidValue;
+  const int hd = C / heads;
+  const size_t smem = sizeof(float) * 2 * 32 * hd;
+  if (smem > 48 * 1024) return cudaErrorInvalidValue;
+  const float alpha =
+      static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(hd)));
+  const dim3 grid(heads, F, (C + 255) / 256);
+  motion_fold_kernel<<<grid, 256, smem, s>>>(kv, wq, mo, C, heads, alpha, wqk, vm);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_motion_attn(const float* q, int64_t ldq, const float* kv, int F, int N,
                                int C, int heads, __half* out, int64_t ldo, cudaStream_t s) {
   const int hd = C / heads;

@@ -78,5 +78,10 @@ cudaError_t launch_motion_kv(const float* motion, const __half* m_kv, int F, int
 // q fp32 (the Mq projection's fp32 accumulators), K/V fp32, out fp16.
 cudaError_t launch_motion_attn(const float* q, int64_t ldq, const float* kv, int F, int N,
                                int C, int heads, __half* out, int64_t ldo, cudaStream_t s);
+// Folded motion cross-attention weights of every frame and head (see
+// motion_fold_kernel): W_qk fp16 [F][C][32 heads] (scores in base 2) and VM
+// fp16 [F][32 heads][C], from K/V (fp32 [F][32][2C]), Wq and Mo (fp16 [C][C]).
+cudaError_t launch_motion_fold(const float* kv, const __half* wq, const __half* mo, int F, int C,
+                               int heads, __half* wqk, __half* vm, cudaStream_t s);
 
 }  // namespace pl

@@ -7,6 +7,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "../../include/pl.h"
 #include "attn.cuh"
@@ -108,7 +109,10 @@ struct pl_ctx {
   __half* qkv;
   __half* attn_o;
   __half* a1;
-  float* qm;                          // fp32 motion queries (Mq accumulators)
+  float* qm;                          // fp32 motion queries (Mq accumulators); on the
+                                      // folded path the fp16 probabilities P [M][32 H]
+  __half* fold_wqk;                   // folded motion path: fp16 [S][16][C][32 H]
+  __half* fold_vm;                    // and fp16 [S][16][32 H][C]
   __half* om;
   __half* out_default;
   pl::DdimCoef coef;
@@ -124,9 +128,11 @@ struct pl_ctx {
     cudaGraphExec_t exec;
     const void* key[64];
     int key_n;
+    int kernels;            // kernel nodes of the captured round
     uint64_t last_use;
   } graphs[2];
   uint64_t graph_tick;
+  int last_round_kernels;   // kernels of the last round run from a capture (-1: none)
   // host path: copy stream, staging-set events, rounds issued
   cudaStream_t copy_stream;
   cudaEvent_t ev_in[2];     // set b's inputs are on the device
@@ -140,6 +146,18 @@ struct pl_ctx {
 };
 
 namespace {
+
+// The motion cross-attention runs folded (scores X W_qk with the softmax in
+// the GEMM epilogue, output P VM) on layers of at least this many tokens per
+// frame. Measured on the 512x512 round (graph-captured, same box, three runs
+// each): 20.12 ms unfolded, 19.75 ms folded at 64x64 only, 19.84 ms folded
+// at 32x32 too (its layers 0.501 -> 0.534 ms: the row kernel there beats the
+// fold, whose W_qk / VM cost grows with C^2); at 16x16 and below forming W_qk
+// and VM costs more than the attention itself.
+constexpr int kFoldMinTokens = 4096;
+bool fold_layer(const pl_config& c, int l) {
+  return c.layer_tokens[l] >= kFoldMinTokens && 16 * c.heads <= c.layer_channels[l];
+}
 
 // Workspace layout; with ctx == nullptr only the size is computed.
 size_t layout(const pl_config& c, pl_ctx* ctx) {
@@ -181,6 +199,12 @@ size_t layout(const pl_config& c, pl_ctx* ctx) {
   uint8_t* qm = take(sizeof(float) * max_nc);
   uint8_t* om = take(sizeof(__half) * max_nc);
   uint8_t* od = take(sizeof(__half) * max_nc);
+  int64_t fold_c = 0;
+  for (int l = 0; l < c.n_layers; ++l)
+    if (fold_layer(c, l) && c.layer_channels[l] > fold_c) fold_c = c.layer_channels[l];
+  const int64_t fold_elems = S * 16 * fold_c * 32 * c.heads;
+  uint8_t* fwqk = fold_elems ? take(sizeof(__half) * fold_elems) : nullptr;
+  uint8_t* fvm = fold_elems ? take(sizeof(__half) * fold_elems) : nullptr;
   if (ctx) {
     ctx->st = reinterpret_cast<pl::DevState*>(st);
     ctx->ring = reinterpret_cast<float*>(ring);
@@ -193,6 +217,8 @@ size_t layout(const pl_config& c, pl_ctx* ctx) {
     ctx->qm = reinterpret_cast<float*>(qm);
     ctx->om = reinterpret_cast<__half*>(om);
     ctx->out_default = reinterpret_cast<__half*>(od);
+    ctx->fold_wqk = reinterpret_cast<__half*>(fwqk);
+    ctx->fold_vm = reinterpret_cast<__half*>(fvm);
   }
   return off;
 }
@@ -261,6 +287,32 @@ pl_status single_gemm(const void* a, int64_t lda, const void* b, int64_t ldb, vo
   return gemm_status(pl::gemm_launch(&gp, s, num_sms()));
 }
 
+// One GEMM per frame f < F with a B of its own: C_f = A_f B_f, where A_f =
+// a + f N lda, B_f = b + f b_stride and C_f = c + f N ldc hold N rows each;
+// up to kGemmMaxProblems frames per launch. softmax32: fp16 output with each
+// 32-column group replaced by its softmax (base-2 logits).
+pl_status frame_gemm(const __half* a, int64_t lda, const __half* b, int64_t ldb, int64_t b_stride,
+                     __half* c, int64_t ldc, int F, int N, int n_cols, int K, bool softmax32,
+                     uint32_t* status, cudaStream_t s) {
+  for (int f0 = 0; f0 < F; f0 += pl::kGemmMaxProblems) {
+    GemmParams gp;
+    std::memset(&gp, 0, sizeof(gp));
+    gp.status = status;
+    const int nf = F - f0 < pl::kGemmMaxProblems ? F - f0 : pl::kGemmMaxProblems;
+    for (int i = 0; i < nf; ++i) {
+      const int64_t f = f0 + i;
+      const int r = pl::gemm_make_problem(&gp.prob[i], a + f * N * lda, lda, b + f * b_stride, ldb,
+                                          c + f * N * ldc, ldc, N, n_cols, K, nullptr, false);
+      if (r) return gemm_status(r);
+      if (softmax32 && pl::gemm_set_softmax32(&gp.prob[i])) return PL_EINVAL;
+    }
+    gp.n_problems = nf;
+    const pl_status r = gemm_status(pl::gemm_launch(&gp, s, num_sms()));
+    if (r) return r;
+  }
+  return PL_OK;
+}
+
 struct RoundArgs {
   const float* new_noise;
   const float* new_motion;
@@ -326,37 +378,74 @@ pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
     if (ar) return ar == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
     uint32_t* status = &ctx->st->status;
     const int Mi = static_cast<int>(M);
-    if (a.attn_out) {
-      // the sub-layer output is wanted: O Wo, then its motion queries
-      __half* a1 = static_cast<__half*>(a.attn_out[l]);
-      r = single_gemm(ctx->attn_o, C, w.w_o, C, a1, C, Mi, C, C, status, s);
-      if (r) return r;
-      r = single_gemm(a1, C, w.m_q, C, ctx->qm, C, Mi, C, C, status, s, /*out_f32=*/true);
-    } else {
-      // motion queries straight from O: O (Wo Mq)
-      r = single_gemm(ctx->attn_o, C, ctx->w_oq[l], C, ctx->qm, C, Mi, C, C, status, s,
-                      /*out_f32=*/true);
-    }
-    if (r) return r;
-    r = from_cuda(pl::launch_motion_attn(ctx->qm, C, ctx->motion_kv[l], F, N, C, H, ctx->om, C, s));
-    if (r) return r;
-    if (ctx->motion_blocks == 2) {
-      // block 2's queries from block 1's output: y1 Mq2 = om (Mo Mq2)
+    if (fold_layer(c, l)) {
+      // motion cross-attention, folded: per frame the scores X W_qk with the
+      // softmax over each head's 32 tokens in the GEMM epilogue (P, fp16, in
+      // the query buffer), then the block output P VM; block 2 takes block 1's
+      // output as its X
+      const int NT = 32 * H;
+      __half* P = reinterpret_cast<__half*>(ctx->qm);
+      const __half* x = ctx->attn_o;
+      const void* wq = ctx->w_oq[l];   // O (Wo Mq)
       if (a.attn_out) {
-        r = single_gemm(ctx->om, C, w.m_o, C, ctx->a1, C, Mi, C, C, status, s);
+        // the sub-layer output is wanted: O Wo, then its motion queries
+        __half* a1 = static_cast<__half*>(a.attn_out[l]);
+        r = single_gemm(ctx->attn_o, C, w.w_o, C, a1, C, Mi, C, C, status, s);
         if (r) return r;
-        r = single_gemm(ctx->a1, C, w.m2_q, C, ctx->qm, C, Mi, C, C, status, s, true);
+        x = a1;
+        wq = w.m_q;
+      }
+      for (int b = 0; b < ctx->motion_blocks; ++b) {
+        const bool second = b == 1;
+        __half* y = b == ctx->motion_blocks - 1 ? out : ctx->om;
+        r = from_cuda(pl::launch_motion_fold(
+            second ? ctx->motion_kv2[l] : ctx->motion_kv[l],
+            static_cast<const __half*>(second ? w.m2_q : wq),
+            static_cast<const __half*>(second ? w.m2_o : w.m_o), F, C, H, ctx->fold_wqk,
+            ctx->fold_vm, s));
+        if (r) return r;
+        r = frame_gemm(x, C, ctx->fold_wqk, NT, static_cast<int64_t>(C) * NT, P, NT, F, N, NT, C,
+                       true, status, s);
+        if (r) return r;
+        r = frame_gemm(P, NT, ctx->fold_vm, C, static_cast<int64_t>(NT) * C, y, C, F, N, C, NT,
+                       false, status, s);
+        if (r) return r;
+        x = y;
+      }
+    } else {
+      if (a.attn_out) {
+        // the sub-layer output is wanted: O Wo, then its motion queries
+        __half* a1 = static_cast<__half*>(a.attn_out[l]);
+        r = single_gemm(ctx->attn_o, C, w.w_o, C, a1, C, Mi, C, C, status, s);
+        if (r) return r;
+        r = single_gemm(a1, C, w.m_q, C, ctx->qm, C, Mi, C, C, status, s, /*out_f32=*/true);
       } else {
-        r = single_gemm(ctx->om, C, ctx->w_oq2[l], C, ctx->qm, C, Mi, C, C, status, s, true);
+        // motion queries straight from O: O (Wo Mq)
+        r = single_gemm(ctx->attn_o, C, ctx->w_oq[l], C, ctx->qm, C, Mi, C, C, status, s,
+                        /*out_f32=*/true);
       }
       if (r) return r;
-      r = from_cuda(pl::launch_motion_attn(ctx->qm, C, ctx->motion_kv2[l], F, N, C, H, ctx->om,
-                                           C, s));
+      r = from_cuda(
+          pl::launch_motion_attn(ctx->qm, C, ctx->motion_kv[l], F, N, C, H, ctx->om, C, s));
+      if (r) return r;
+      if (ctx->motion_blocks == 2) {
+        // block 2's queries from block 1's output: y1 Mq2 = om (Mo Mq2)
+        if (a.attn_out) {
+          r = single_gemm(ctx->om, C, w.m_o, C, ctx->a1, C, Mi, C, C, status, s);
+          if (r) return r;
+          r = single_gemm(ctx->a1, C, w.m2_q, C, ctx->qm, C, Mi, C, C, status, s, true);
+        } else {
+          r = single_gemm(ctx->om, C, ctx->w_oq2[l], C, ctx->qm, C, Mi, C, C, status, s, true);
+        }
+        if (r) return r;
+        r = from_cuda(pl::launch_motion_attn(ctx->qm, C, ctx->motion_kv2[l], F, N, C, H, ctx->om,
+                                             C, s));
+        if (r) return r;
+      }
+      const void* w_last = ctx->motion_blocks == 2 ? w.m2_o : w.m_o;
+      r = single_gemm(ctx->om, C, w_last, C, out, C, Mi, C, C, status, s);
       if (r) return r;
     }
-    const void* w_last = ctx->motion_blocks == 2 ? w.m2_o : w.m_o;
-    r = single_gemm(ctx->om, C, w_last, C, out, C, Mi, C, C, status, s);
-    if (r) return r;
   }
   if (a.layer_events && c.n_layers > 0 &&
       cudaEventRecord(a.layer_events[c.n_layers], s) != cudaSuccess)
@@ -387,6 +476,22 @@ void drop_slot(pl_ctx::GraphSlot& g) {
   g.exec = nullptr;
   g.graph = nullptr;
   g.key_n = 0;
+  g.kernels = 0;
+}
+
+// kernel nodes of a captured graph (-1 when the graph cannot be read)
+int count_kernel_nodes(cudaGraph_t g) {
+  size_t n = 0;
+  if (cudaGraphGetNodes(g, nullptr, &n) != cudaSuccess) return -1;
+  std::vector<cudaGraphNode_t> nodes(n);
+  if (n && cudaGraphGetNodes(g, nodes.data(), &n) != cudaSuccess) return -1;
+  int k = 0;
+  for (size_t i = 0; i < n; ++i) {
+    cudaGraphNodeType t;
+    if (cudaGraphNodeGetType(nodes[i], &t) != cudaSuccess) return -1;
+    if (t == cudaGraphNodeTypeKernel) ++k;
+  }
+  return k;
 }
 
 void drop_graph(pl_ctx* ctx) {
@@ -446,7 +551,7 @@ const char* pl_status_string(int status) {
   }
 }
 
-int pl_abi_version(void) { return 2; }
+int pl_abi_version(void) { return 3; }
 
 pl_status pl_gemm_f16(const void* a, int64_t lda, const void* b, int64_t ldb, void* c,
                       int64_t ldc, int M, int N, int K, void* stream) {
@@ -731,6 +836,7 @@ pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_
   ctx->sessions = cfg->sessions > 0 ? cfg->sessions : 1;
   ctx->capacity = 1 + cfg->append_cap;
   ctx->motion_blocks = cfg->motion_blocks == 2 ? 2 : 1;
+  ctx->last_round_kernels = -1;
   ctx->frame_elems = static_cast<int64_t>(cfg->latent_c) * cfg->latent_h * cfg->latent_w;
   ctx->ws = static_cast<uint8_t*>(workspace);
   ctx->ws_bytes = workspace_bytes;
@@ -935,10 +1041,12 @@ pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_
       return PL_ECUDA;
     }
     slot->graph = g;
+    slot->kernels = count_kernel_nodes(g);
     std::memcpy(slot->key, key, sizeof(const void*) * kn);
     slot->key_n = kn;
   }
   slot->last_use = ++ctx->graph_tick;
+  ctx->last_round_kernels = slot->kernels;
   return from_cuda(cudaGraphLaunch(slot->exec, s));
 }
 
@@ -1202,6 +1310,13 @@ pl_status pl_set_profiling(pl_ctx* ctx, int on) {
   if (!ctx) return PL_EINVAL;
   ctx->profile = on != 0;
   ctx->prof_valid = false;
+  return PL_OK;
+}
+
+pl_status pl_round_kernel_count(const pl_ctx* ctx, int* count) {
+  if (!ctx || !count) return PL_EINVAL;
+  if (ctx->last_round_kernels < 0) return PL_ESTATE;
+  *count = ctx->last_round_kernels;
   return PL_OK;
 }
 

@@ -577,6 +577,13 @@ pl_status pl_get_device_status(pl_ctx* ctx, void* stream);
 pl_status pl_set_profiling(pl_ctx* ctx, int on);
 pl_status pl_get_layer_ms(pl_ctx* ctx, float* ms_out, int n);
 
+/* Kernels in the captured graph of the latest round that ran from a capture
+ * (pl_stream_round with profiling off, or pl_stream_round_host): every
+ * kernel of this library that one round launches, counted from the graph's
+ * nodes when it was captured. *count (host); PL_ESTATE when no round has run
+ * from a capture yet. */
+pl_status pl_round_kernel_count(const pl_ctx* ctx, int* count);
+
 /* Checkpoint and resume of the streams' state (no counterpart in the pages,
  * which pause and reset a stream but do not resume one; the state is small
  * and device-resident, so it is the natural unit to save).

@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings_and_abi():
     import denoise_step_b200 as P
-    assert P.lib.pl_abi_version() == 2
+    assert P.lib.pl_abi_version() == 3
     for s in range(8):
         assert P.lib.pl_status_string(s)
     assert P.lib.pl_status_string(99) == b"unknown status"
@@ -167,6 +167,8 @@ def test_state_and_profiling_calls_validate_their_arguments():
     assert P.lib.pl_set_profiling(None, 1) == P.PL_EINVAL
     buf = (C.c_float * 4)()
     assert P.lib.pl_get_layer_ms(None, buf, 4) == P.PL_EINVAL
+    k = C.c_int()
+    assert P.lib.pl_round_kernel_count(None, C.byref(k)) == P.PL_EINVAL
 
 
 def test_round_before_init_is_a_state_error():

@@ -218,10 +218,11 @@ def test_full_geometry_rounds_spot_checked(P):
     st.close()
 
 
-def _block2_logit_std(h, w, bank, motion, heads=8):
-    """Std of the second motion block's logits (fp64, oracle inputs)."""
+def _block2_logit_std(h, w, bank, motion, heads=8, rows=None):
+    """Std of the second motion block's logits (fp64, oracle inputs; `rows`:
+    those query rows only)."""
     tok = O.motion_tokens(motion)
-    y1 = O.motion_xattn_frame(O.ref_attention_frame(h, w, bank, heads), tok, w, heads)
+    y1 = O.motion_xattn_frame(O.ref_attention_frame(h, w, bank, heads, rows=rows), tok, w, heads)
     q = y1 @ np.asarray(w["mq2"], np.float64)
     k = tok @ np.asarray(w["mk2"], np.float64)
     hd = q.shape[1] // heads
@@ -280,6 +281,67 @@ def test_two_motion_blocks_tiny_rounds(P, sublayer):
             if sublayer:
                 want_a = O.ref_attention_frame(hidden[0][f], case.w[0], bank, 8)
                 mx, mean, rel = attn_errors(host(attn_out[0])[f], want_a)
+                assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (r, f, mx, mean, rel)
+        want_x0 = orc.step_and_pop(eps)
+        _, _, want_flags = orc.check_bank(mot)
+        orc.rounds += 1
+        assert np.max(np.abs(host(out) - want_x0)) <= DDIM_ABS, r
+        assert list(host(flags)) == want_flags, r
+    assert st.device_status() == 0
+    st.close()
+
+
+@pytest.mark.parametrize("sublayer", [False, True])
+def test_two_motion_blocks_level64_folded(P, sublayer):
+    # At 64x64 the round runs the motion cross-attention folded: per frame the
+    # scores X W_qk (W_qk = Wq K^T / sqrt(hd), fp16) with the softmax over each
+    # head's 32 tokens in the GEMM epilogue, then the block output P VM (VM =
+    # V Mo per head). Two blocks, block 2 queried by block 1's fp16 output,
+    # two rounds (bank x2 in round 2), sampled rows of frames 0 and 9, the
+    # gates of the tiny two-block rounds; with `sublayer` Wo, Mq and Mq2 are
+    # applied separately and the reference-attention output is checked too
+    case = Case(S.SEEDS["tiny"] + 11, [("m", 64, 320)], 64, 64, 3.0)
+    case.w[0].update(S.motion_block_weights(case.seed, "m", 320, 2, np.float16))
+    cfg = P.make_config((64, 64), [(4096, 320)], motion_blocks=2)
+    st = P.Stream(cfg)
+    pw = [pack_weights(w) for w in case.w]
+    drive0 = S.normal(case.seed, "drive0", (512,), 1.0, np.float32)
+    st.bank_init(pw, [dev(f) for f in case.ref_feats], [dev(a) for an in case.anchors for a in an],
+                 dev(case.ref_motion), dev(drive0), dev(case.ref_latent), dev(case.prefill_eps))
+    orc = O.PyramidStream(case.ref_latent, case.prefill_eps, case.ref_motion, drive0,
+                          state_dtype=np.float32)
+    stream = torch.cuda.Stream()
+    out = torch.empty((4, 4, 64, 64), dtype=torch.float32, device="cuda")
+    flags = torch.zeros(4, dtype=torch.uint8, device="cuda")
+    layer_out = [torch.empty((16, 4096, 320), dtype=torch.float16, device="cuda")]
+    attn_out = [torch.empty_like(layer_out[0])] if sublayer else None
+    rows = np.unique(S.uniform_int(case.seed, "rows", 24, 4096))
+    for r in (1, 2):
+        hidden, noise, eps = case.round_inputs(r)
+        mot = case.next_motion(r)
+        d_in = ([dev(h) for h in hidden], dev(noise), dev(mot), dev(eps))
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            st.round(d_in[1], d_in[2], d_in[0], d_in[3], out, flags, layer_out, stream=stream,
+                     attn_out=attn_out)
+        stream.synchronize()
+        n_kv = 1 + orc.appends
+        orc.append(noise, mot)
+        bm = orc.batch_motion()
+        got = host(layer_out[0])
+        for f in (0, 9):
+            bank = _kv_bank(case, 0, n_kv)
+            want = O.layer_forward_frame(hidden[0][f], case.w[0], bank, O.motion_tokens(bm[f]), 8,
+                                         rows=rows, motion_blocks=2)
+            mx, mean, rel = attn_errors(got[f][rows], want)
+            g = scaled_gates(want)
+            kappa = max(1.0, _block2_logit_std(hidden[0][f], case.w[0], bank, bm[f], rows=rows))
+            assert mx <= ATTN_MAX_ABS * g * kappa and mean <= ATTN_MEAN_ABS * g * kappa, \
+                (r, f, mx, mean, rel, g, kappa)
+            assert rel < 2e-3 * kappa, (r, f, rel, kappa)
+            if sublayer:
+                want_a = O.ref_attention_frame(hidden[0][f], case.w[0], bank, 8, rows=rows)
+                mx, mean, rel = attn_errors(host(attn_out[0])[f][rows], want_a)
                 assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (r, f, mx, mean, rel)
         want_x0 = orc.step_and_pop(eps)
         _, _, want_flags = orc.check_bank(mot)

@@ -30,13 +30,14 @@ def P():
 class Session:
     """Seeded inputs of one stream; the weights are the model's (shared)."""
 
-    def __init__(self, seed, walk_sigma, weights):
-        self.seed, self.w = seed, weights
-        self.ref_feats = [S.bank_features(seed, n, 0, s * s, C) for n, s, C in LAYERS]
-        self.anchors = [[S.bank_features(seed, n, a, s * s, C) for n, s, C in LAYERS]
+    def __init__(self, seed, walk_sigma, weights, layers=LAYERS, hw=(H, W)):
+        self.seed, self.w, self.layers, self.hw = seed, weights, layers, hw
+        h, w = hw
+        self.ref_feats = [S.bank_features(seed, n, 0, s * s, C) for n, s, C in layers]
+        self.anchors = [[S.bank_features(seed, n, a, s * s, C) for n, s, C in layers]
                         for a in range(1, 4)]
-        self.ref_latent = S.normal(seed, "ref_latent", (4, H, W), 1.0, np.float32)
-        self.prefill_eps = S.normal(seed, "prefill_eps", (12, 4, H, W), 1.0, np.float32)
+        self.ref_latent = S.normal(seed, "ref_latent", (4, h, w), 1.0, np.float32)
+        self.prefill_eps = S.normal(seed, "prefill_eps", (12, 4, h, w), 1.0, np.float32)
         self.ref_motion = S.normal(seed, "walk/e0", (512,), 1.0, np.float32)
         self.drive0 = S.normal(seed, "drive0", (512,), 1.0, np.float32)
         self.walk_sigma = walk_sigma
@@ -54,29 +55,32 @@ class Session:
         return out
 
     def round_inputs(self, r):
-        hidden = [S.layer_hidden(self.seed, n, r, 16, s * s, C) for n, s, C in LAYERS]
-        noise = S.normal(self.seed, f"noise{r}", (4, 4, H, W), 1.0, np.float32)
-        eps = S.normal(self.seed, f"eps{r}", (16, 4, H, W), 1.0, np.float32)
+        h, w = self.hw
+        hidden = [S.layer_hidden(self.seed, n, r, 16, s * s, C) for n, s, C in self.layers]
+        noise = S.normal(self.seed, f"noise{r}", (4, 4, h, w), 1.0, np.float32)
+        eps = S.normal(self.seed, f"eps{r}", (16, 4, h, w), 1.0, np.float32)
         return hidden, noise, eps
 
     def kv_bank(self, li, n_entries):
         return [self.ref_feats[li]] + [self.anchors[a][li] for a in range(n_entries - 1)]
 
 
-def _sessions(sigmas):
+def _sessions(sigmas, layers=LAYERS, hw=(H, W)):
     base = S.SEEDS["tiny"]
-    weights = [layer_weights_np(base, n, C) for n, _, C in LAYERS]
-    return [Session(base + 100 * (z + 1), sig, weights) for z, sig in enumerate(sigmas)]
+    weights = [layer_weights_np(base, n, C) for n, _, C in layers]
+    return [Session(base + 100 * (z + 1), sig, weights, layers, hw)
+            for z, sig in enumerate(sigmas)]
 
 
 def _ctx(P, sess):
     """One context serving `sess` (leading session dimension on every input)."""
-    cfg = P.make_config((H, W), [(s * s, C) for _, s, C in LAYERS], sessions=len(sess))
+    layers = sess[0].layers
+    cfg = P.make_config(sess[0].hw, [(s * s, C) for _, s, C in layers], sessions=len(sess))
     st = P.Stream(cfg)
     pw = [pack_weights(w) for w in sess[0].w]
     stack = lambda xs: dev(np.stack(xs))
-    ref = [stack([z.ref_feats[li] for z in sess]) for li in range(len(LAYERS))]
-    anc = [stack([z.anchors[a][li] for z in sess]) for a in range(3) for li in range(len(LAYERS))]
+    ref = [stack([z.ref_feats[li] for z in sess]) for li in range(len(layers))]
+    anc = [stack([z.anchors[a][li] for z in sess]) for a in range(3) for li in range(len(layers))]
     st.bank_init(pw, ref, anc, stack([z.ref_motion for z in sess]),
                  stack([z.drive0 for z in sess]), stack([z.ref_latent for z in sess]),
                  stack([z.prefill_eps for z in sess]))
@@ -85,15 +89,16 @@ def _ctx(P, sess):
 
 def _run_round(st, sess, inputs, stream):
     Sn = len(sess)
+    layers, (h, w) = sess[0].layers, sess[0].hw
     stack = lambda xs: dev(np.stack(xs))
-    d_hidden = [stack([inp[0][li] for inp in inputs]) for li in range(len(LAYERS))]
+    d_hidden = [stack([inp[0][li] for inp in inputs]) for li in range(len(layers))]
     d_noise = stack([inp[1] for inp in inputs])
     d_mot = stack([inp[3] for inp in inputs])
     d_eps = stack([inp[2] for inp in inputs])
-    out = torch.empty((Sn, 4, 4, H, W), dtype=torch.float32, device="cuda")
+    out = torch.empty((Sn, 4, 4, h, w), dtype=torch.float32, device="cuda")
     flags = torch.zeros((Sn, 4), dtype=torch.uint8, device="cuda")
     layer_out = [torch.empty((Sn, 16, s * s, C), dtype=torch.float16, device="cuda")
-                 for _, s, C in LAYERS]
+                 for _, s, C in layers]
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         st.round(d_noise, d_mot, d_hidden, d_eps, out, flags, layer_out, stream=stream)
@@ -146,8 +151,14 @@ def test_sessions_match_their_oracles(P):
     st.close()
 
 
-def test_batched_sessions_equal_single_streams(P):
-    sess = _sessions([3.0, 0.5])
+@pytest.mark.parametrize("geometry", ["8x8", "64x64"])
+def test_batched_sessions_equal_single_streams(P, geometry):
+    # at 64x64 the motion cross-attention runs folded, its per-frame GEMMs in
+    # one launch per 16 frames (two launches for the batched pair)
+    if geometry == "8x8":
+        sess = _sessions([3.0, 0.5])
+    else:
+        sess = _sessions([3.0, 0.5], [("d00", 64, 320)], (64, 64))
     batched = _ctx(P, sess)
     singles = [_ctx(P, [z]) for z in sess]
     stream = torch.cuda.Stream()
@@ -161,7 +172,7 @@ def test_batched_sessions_equal_single_streams(P):
             out_s, flags_s, lo_s = _run_round(single, [z], [inputs[zi]], stream)
             assert np.array_equal(out_b[zi], out_s[0]), (r, zi)
             assert np.array_equal(flags_b[zi], flags_s[0]), (r, zi)
-            for li in range(len(LAYERS)):
+            for li in range(len(sess[0].layers)):
                 assert np.array_equal(lo_b[li][zi], lo_s[li][0]), (r, zi, li)
             assert batched.state(session=zi) == single.state(), (r, zi)
     batched.close()

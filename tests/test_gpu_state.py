@@ -142,5 +142,14 @@ def test_profiled_round_matches_the_graph_round(P):
     b.set_profiling(False)
     with pytest.raises(P.PLError):
         b.layer_ms()
+    with pytest.raises(P.PLError):
+        b.round_kernels()                     # b has run no round from a capture
+    # a ran from its captured graph: the same kernel count every round, at
+    # least the reference attention, its projection and the motion sub-layer
+    # per layer plus the ring, DDIM and bank-check kernels
+    k = a.round_kernels()
+    assert k >= 3 * len(LAYERS) + 4, k
+    _run(P, a, seed, 3, stream)
+    assert a.round_kernels() == k
     a.close()
     b.close()
