@@ -1350,14 +1350,38 @@ __global__ void __launch_bounds__(256) motion_fold_kernel(const float* __restric
   const float* sv = skv + 32 * hd;
   const int c = blockIdx.z * blockDim.x + threadIdx.x;
   if (c >= C) return;
+  // eight head channels at a time: K[t][d0..d0+7] and V[t][..] as two 16-byte
+  // broadcast reads each, feeding 8 fmas (hd is a multiple of 8)
   float acc[32];
 #pragma unroll
   for (int t = 0; t < 32; ++t) acc[t] = 0.f;
   const __half* wrow = wq + static_cast<int64_t>(c) * C + h * hd;
-  for (int d = 0; d < hd; ++d) {
-    const float w = __half2float(wrow[d]);
+  for (int d0 = 0; d0 < hd; d0 += 8) {
+    float w[8];
+    {
+      const uint4 u = *reinterpret_cast<const uint4*>(wrow + d0);
+      const __half2* hv = reinterpret_cast<const __half2*>(&u);
 #pragma unroll
-    for (int t = 0; t < 32; ++t) acc[t] = fmaf(w, sk[t * hd + d], acc[t]);
+      for (int j = 0; j < 4; ++j) {
+        const float2 f2 = __half22float2(hv[j]);
+        w[2 * j] = f2.x;
+        w[2 * j + 1] = f2.y;
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      const float4 k0 = *reinterpret_cast<const float4*>(sk + t * hd + d0);
+      const float4 k1 = *reinterpret_cast<const float4*>(sk + t * hd + d0 + 4);
+      float a_ = acc[t];
+      a_ = fmaf(w[0], k0.x, a_);
+      a_ = fmaf(w[1], k0.y, a_);
+      a_ = fmaf(w[2], k0.z, a_);
+      a_ = fmaf(w[3], k0.w, a_);
+      a_ = fmaf(w[4], k1.x, a_);
+      a_ = fmaf(w[5], k1.y, a_);
+      a_ = fmaf(w[6], k1.z, a_);
+      acc[t] = fmaf(w[7], k1.w, a_);
+    }
   }
   __half* o = wqk + (static_cast<int64_t>(f) * C + c) * NT + 32 * h;
 #pragma unroll
@@ -1365,10 +1389,24 @@ __global__ void __launch_bounds__(256) motion_fold_kernel(const float* __restric
     *reinterpret_cast<__half2*>(o + t) = __floats2half2_rn(alpha * acc[t], alpha * acc[t + 1]);
 #pragma unroll
   for (int t = 0; t < 32; ++t) acc[t] = 0.f;
-  for (int d = 0; d < hd; ++d) {
-    const float m = __half2float(mo[static_cast<int64_t>(h * hd + d) * C + c]);
+  for (int d0 = 0; d0 < hd; d0 += 8) {
+    float m[8];
 #pragma unroll
-    for (int t = 0; t < 32; ++t) acc[t] = fmaf(sv[t * hd + d], m, acc[t]);
+    for (int j = 0; j < 8; ++j) m[j] = __half2float(mo[static_cast<int64_t>(h * hd + d0 + j) * C + c]);
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      const float4 v0 = *reinterpret_cast<const float4*>(sv + t * hd + d0);
+      const float4 v1 = *reinterpret_cast<const float4*>(sv + t * hd + d0 + 4);
+      float a_ = acc[t];
+      a_ = fmaf(v0.x, m[0], a_);
+      a_ = fmaf(v0.y, m[1], a_);
+      a_ = fmaf(v0.z, m[2], a_);
+      a_ = fmaf(v0.w, m[3], a_);
+      a_ = fmaf(v1.x, m[4], a_);
+      a_ = fmaf(v1.y, m[5], a_);
+      a_ = fmaf(v1.z, m[6], a_);
+      acc[t] = fmaf(v1.w, m[7], a_);
+    }
   }
   __half* v = vm + (static_cast<int64_t>(f) * NT + 32 * h) * C + c;
 #pragma unroll
@@ -1377,8 +1415,9 @@ __global__ void __launch_bounds__(256) motion_fold_kernel(const float* __restric
 
 cudaError_t launch_motion_fold(const float* kv, const __half* wq, const __half* mo, int F, int C,
                                int heads, __half* wqk, __half* vm, cudaStream_t s) {
-  if (heads < 1 || C % heads) return cudaErrorInvalidValue;
+  if (heads < 1 || C % heads || C % 8) return cudaErrorInvalidValue;
   const int hd = C / heads;
+  if (hd % 8 || (reinterpret_cast<uintptr_t>(wq) & 15)) return cudaErrorInvalidValue;
   const size_t smem = sizeof(float) * 2 * 32 * hd;
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
   const float alpha =
