@@ -150,11 +150,11 @@ namespace {
 // The motion cross-attention runs folded (scores X W_qk with the softmax in
 // the GEMM epilogue, output P VM) on layers of at least this many tokens per
 // frame. Measured on the 512x512 round (graph-captured, same box, three runs
-// each): 20.12 ms unfolded, 19.75 ms folded at 64x64 only, 19.84 ms folded
-// at 32x32 too (its layers 0.501 -> 0.534 ms: the row kernel there beats the
-// fold, whose W_qk / VM cost grows with C^2); at 16x16 and below forming W_qk
-// and VM costs more than the attention itself.
-constexpr int kFoldMinTokens = 4096;
+// each): 20.12 ms unfolded, 19.75 ms folded at 64x64; with the fold kernel
+// reading eight head channels per step, 19.84 ms folded at 64x64 against
+// 19.74 ms at 32x32 too (its layers 0.501 -> 0.475 ms). At 16x16 and below
+// forming W_qk and VM (which grows with C^2) costs more than the attention.
+constexpr int kFoldMinTokens = 1024;
 bool fold_layer(const pl_config& c, int l) {
   return c.layer_tokens[l] >= kFoldMinTokens && 16 * c.heads <= c.layer_channels[l];
 }
