@@ -106,15 +106,22 @@ struct pl_ctx {
   float* motion_kv2[PL_MAX_LAYERS];  // second motion block's, as motion_kv
   __half* w_oq[PL_MAX_LAYERS];        // fp16 [C][C] = Wo Mq
   __half* w_oq2[PL_MAX_LAYERS];       // fp16 [C][C] = Mo Mq2 (two motion blocks)
-  __half* qkv;
-  __half* attn_o;
-  __half* a1;
-  float* qm;                          // fp32 motion queries (Mq accumulators); on the
-                                      // folded path the fp16 probabilities P [M][32 H]
-  __half* fold_wqk;                   // folded motion path: fp16 [S][16][C][32 H]
-  __half* fold_vm;                    // and fp16 [S][16][32 H][C]
-  __half* om;
-  __half* out_default;
+  // per-layer scratch, two sets: the round runs even layers on its stream
+  // with set 0 and odd layers on a second stream with set 1 (the layers are
+  // independent: each has its own hidden input and output)
+  struct Scratch {
+    __half* qkv;
+    __half* attn_o;
+    __half* a1;
+    float* qm;          // fp32 motion queries (Mq accumulators); on the folded
+                        // path the fp16 probabilities P [M][32 H]
+    __half* om;
+    __half* out_default;
+    __half* fold_wqk;   // folded motion path: fp16 [S][16][C][32 H]
+    __half* fold_vm;    // and fp16 [S][16][32 H][C]
+  } sc[2];
+  cudaStream_t side;               // the round's second stream (odd layers)
+  cudaEvent_t ev_fork, ev_join;    // its fork after the ring push, its join
   pl::DdimCoef coef;
   bool initialised;
   bool have_anchors;
@@ -193,32 +200,37 @@ size_t layout(const pl_config& c, pl_ctx* ctx) {
     }
     if (S * 16 * N * C > max_nc) max_nc = S * 16 * N * C;
   }
-  uint8_t* qkv = take(sizeof(__half) * 3 * max_nc);
-  uint8_t* ao = take(sizeof(__half) * max_nc);
-  uint8_t* a1 = take(sizeof(__half) * max_nc);
-  uint8_t* qm = take(sizeof(float) * max_nc);
-  uint8_t* om = take(sizeof(__half) * max_nc);
-  uint8_t* od = take(sizeof(__half) * max_nc);
   int64_t fold_c = 0;
   for (int l = 0; l < c.n_layers; ++l)
     if (fold_layer(c, l) && c.layer_channels[l] > fold_c) fold_c = c.layer_channels[l];
   const int64_t fold_elems = S * 16 * fold_c * 32 * c.heads;
-  uint8_t* fwqk = fold_elems ? take(sizeof(__half) * fold_elems) : nullptr;
-  uint8_t* fvm = fold_elems ? take(sizeof(__half) * fold_elems) : nullptr;
+  for (int k = 0; k < 2; ++k) {
+    uint8_t* qkv = take(sizeof(__half) * 3 * max_nc);
+    uint8_t* ao = take(sizeof(__half) * max_nc);
+    uint8_t* a1 = take(sizeof(__half) * max_nc);
+    uint8_t* qm = take(sizeof(float) * max_nc);
+    uint8_t* om = take(sizeof(__half) * max_nc);
+    uint8_t* od = take(sizeof(__half) * max_nc);
+    uint8_t* fwqk = fold_elems ? take(sizeof(__half) * fold_elems) : nullptr;
+    uint8_t* fvm = fold_elems ? take(sizeof(__half) * fold_elems) : nullptr;
+    if (ctx) {
+      pl_ctx::Scratch& x = ctx->sc[k];
+      x.qkv = reinterpret_cast<__half*>(qkv);
+      x.attn_o = reinterpret_cast<__half*>(ao);
+      x.a1 = reinterpret_cast<__half*>(a1);
+      x.qm = reinterpret_cast<float*>(qm);
+      x.om = reinterpret_cast<__half*>(om);
+      x.out_default = reinterpret_cast<__half*>(od);
+      x.fold_wqk = reinterpret_cast<__half*>(fwqk);
+      x.fold_vm = reinterpret_cast<__half*>(fvm);
+    }
+  }
   if (ctx) {
     ctx->st = reinterpret_cast<pl::DevState*>(st);
     ctx->ring = reinterpret_cast<float*>(ring);
     ctx->slot_motion = reinterpret_cast<float*>(sm);
     ctx->batch_motion = reinterpret_cast<float*>(bm);
     ctx->bank = reinterpret_cast<float*>(bank);
-    ctx->qkv = reinterpret_cast<__half*>(qkv);
-    ctx->attn_o = reinterpret_cast<__half*>(ao);
-    ctx->a1 = reinterpret_cast<__half*>(a1);
-    ctx->qm = reinterpret_cast<float*>(qm);
-    ctx->om = reinterpret_cast<__half*>(om);
-    ctx->out_default = reinterpret_cast<__half*>(od);
-    ctx->fold_wqk = reinterpret_cast<__half*>(fwqk);
-    ctx->fold_vm = reinterpret_cast<__half*>(fvm);
   }
   return off;
 }
@@ -325,6 +337,126 @@ struct RoundArgs {
   cudaEvent_t* layer_events;   // when non-null: [n_layers + 1] recorded around the layers
 };
 
+// Enqueue layer l of a round on `s` with scratch set `sc`.
+pl_status enqueue_layer(pl_ctx* ctx, const RoundArgs& a, int l, const pl_ctx::Scratch& sc,
+                        cudaStream_t s) {
+  const pl_config& c = ctx->cfg;
+  const int S = ctx->sessions;
+  const int F = 16 * S;   // the batches of all sessions, session-major
+  pl_status r = PL_OK;
+  const int N = c.layer_tokens[l], C = c.layer_channels[l], H = c.heads, hd = C / H;
+  const int64_t M = static_cast<int64_t>(F) * N;
+  const pl_layer_weights& w = ctx->w[l];
+  __half* out = a.layer_out ? static_cast<__half*>(a.layer_out[l]) : sc.out_default;
+  r = from_cuda(pl::launch_motion_kv(ctx->batch_motion, static_cast<const __half*>(w.m_kv), F,
+                                     C, ctx->motion_kv[l], s));
+  if (r) return r;
+  if (ctx->motion_blocks == 2) {
+    r = from_cuda(pl::launch_motion_kv(ctx->batch_motion, static_cast<const __half*>(w.m2_kv),
+                                       F, C, ctx->motion_kv2[l], s));
+    if (r) return r;
+  }
+  r = single_gemm(a.hidden[l], C, w.w_qkv, 3 * C, sc.qkv, 3 * C, static_cast<int>(M), 3 * C,
+                  C, &ctx->st->status, s);
+  if (r) return r;
+  // own K/V per frame; bank entry b of session z for the frames of session z
+  AttnSegHost segs[1 + PL_MAX_BANK];
+  segs[0] = {sc.qkv + C, sc.qkv + 2 * C, N, 3ll * C, static_cast<int64_t>(N) * 3 * C};
+  const int nb = ctx->have_anchors ? ctx->capacity : 1;
+  for (int b = 0; b < nb; ++b) {
+    const __half* kv = ctx->bank_kv[l] + static_cast<int64_t>(b) * N * 2 * C;
+    segs[1 + b] = {kv, kv + C, N, 2ll * C, 0};
+    if (S > 1) {
+      segs[1 + b].frame_stride = static_cast<int64_t>(ctx->capacity) * N * 2 * C;
+      segs[1 + b].n_blocks = S;
+      segs[1 + b].frame_div = 16;
+    }
+  }
+  AttnParams ap;
+  int ar = pl::attn_make_params(&ap, sc.qkv, 3ll * C, static_cast<int64_t>(N) * 3 * C, segs,
+                                1 + nb, F, N, H, hd, sc.attn_o, C,
+                                static_cast<int64_t>(N) * C);
+  if (ar) return ar == 1 ? PL_EINVAL : PL_ECUDA;
+  ap.n_fixed = 2;
+  ap.n_extra = ctx->have_anchors ? &ctx->st->appends : nullptr;
+  ap.extra_div = 16;
+  ap.extra_stride = static_cast<int>(sizeof(pl::DevState) / sizeof(int32_t));
+  ap.status = &ctx->st->status;
+  ar = pl::attn_launch(ap, hd, s);
+  if (ar) return ar == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
+  uint32_t* status = &ctx->st->status;
+  const int Mi = static_cast<int>(M);
+  if (fold_layer(c, l)) {
+    // motion cross-attention, folded: per frame the scores X W_qk with the
+    // softmax over each head's 32 tokens in the GEMM epilogue (P, fp16, in
+    // the query buffer), then the block output P VM; block 2 takes block 1's
+    // output as its X
+    const int NT = 32 * H;
+    __half* P = reinterpret_cast<__half*>(sc.qm);
+    const __half* x = sc.attn_o;
+    const void* wq = ctx->w_oq[l];   // O (Wo Mq)
+    if (a.attn_out) {
+      // the sub-layer output is wanted: O Wo, then its motion queries
+      __half* a1 = static_cast<__half*>(a.attn_out[l]);
+      r = single_gemm(sc.attn_o, C, w.w_o, C, a1, C, Mi, C, C, status, s);
+      if (r) return r;
+      x = a1;
+      wq = w.m_q;
+    }
+    for (int b = 0; b < ctx->motion_blocks; ++b) {
+      const bool second = b == 1;
+      __half* y = b == ctx->motion_blocks - 1 ? out : sc.om;
+      r = from_cuda(pl::launch_motion_fold(
+          second ? ctx->motion_kv2[l] : ctx->motion_kv[l],
+          static_cast<const __half*>(second ? w.m2_q : wq),
+          static_cast<const __half*>(second ? w.m2_o : w.m_o), F, C, H, sc.fold_wqk,
+          sc.fold_vm, s));
+      if (r) return r;
+      r = frame_gemm(x, C, sc.fold_wqk, NT, static_cast<int64_t>(C) * NT, P, NT, F, N, NT, C,
+                     true, status, s);
+      if (r) return r;
+      r = frame_gemm(P, NT, sc.fold_vm, C, static_cast<int64_t>(NT) * C, y, C, F, N, C, NT,
+                     false, status, s);
+      if (r) return r;
+      x = y;
+    }
+  } else {
+    if (a.attn_out) {
+      // the sub-layer output is wanted: O Wo, then its motion queries
+      __half* a1 = static_cast<__half*>(a.attn_out[l]);
+      r = single_gemm(sc.attn_o, C, w.w_o, C, a1, C, Mi, C, C, status, s);
+      if (r) return r;
+      r = single_gemm(a1, C, w.m_q, C, sc.qm, C, Mi, C, C, status, s, /*out_f32=*/true);
+    } else {
+      // motion queries straight from O: O (Wo Mq)
+      r = single_gemm(sc.attn_o, C, ctx->w_oq[l], C, sc.qm, C, Mi, C, C, status, s,
+                      /*out_f32=*/true);
+    }
+    if (r) return r;
+    r = from_cuda(
+        pl::launch_motion_attn(sc.qm, C, ctx->motion_kv[l], F, N, C, H, sc.om, C, s));
+    if (r) return r;
+    if (ctx->motion_blocks == 2) {
+      // block 2's queries from block 1's output: y1 Mq2 = om (Mo Mq2)
+      if (a.attn_out) {
+        r = single_gemm(sc.om, C, w.m_o, C, sc.a1, C, Mi, C, C, status, s);
+        if (r) return r;
+        r = single_gemm(sc.a1, C, w.m2_q, C, sc.qm, C, Mi, C, C, status, s, true);
+      } else {
+        r = single_gemm(sc.om, C, ctx->w_oq2[l], C, sc.qm, C, Mi, C, C, status, s, true);
+      }
+      if (r) return r;
+      r = from_cuda(pl::launch_motion_attn(sc.qm, C, ctx->motion_kv2[l], F, N, C, H, sc.om,
+                                           C, s));
+      if (r) return r;
+    }
+    const void* w_last = ctx->motion_blocks == 2 ? w.m2_o : w.m_o;
+    r = single_gemm(sc.om, C, w_last, C, out, C, Mi, C, C, status, s);
+    if (r) return r;
+  }
+  return PL_OK;
+}
+
 // Enqueue one whole round on `s` (also used under stream capture).
 pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
   const pl_config& c = ctx->cfg;
@@ -334,119 +466,28 @@ pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
                                                ctx->batch_motion, a.new_noise, a.new_motion,
                                                ctx->frame_elems, S, s));
   if (r) return r;
-  for (int l = 0; l < c.n_layers; ++l) {
-    if (a.layer_events && cudaEventRecord(a.layer_events[l], s) != cudaSuccess) return PL_ECUDA;
-    const int N = c.layer_tokens[l], C = c.layer_channels[l], H = c.heads, hd = C / H;
-    const int64_t M = static_cast<int64_t>(F) * N;
-    const pl_layer_weights& w = ctx->w[l];
-    __half* out = a.layer_out ? static_cast<__half*>(a.layer_out[l]) : ctx->out_default;
-    r = from_cuda(pl::launch_motion_kv(ctx->batch_motion, static_cast<const __half*>(w.m_kv), F,
-                                       C, ctx->motion_kv[l], s));
-    if (r) return r;
-    if (ctx->motion_blocks == 2) {
-      r = from_cuda(pl::launch_motion_kv(ctx->batch_motion, static_cast<const __half*>(w.m2_kv),
-                                         F, C, ctx->motion_kv2[l], s));
-      if (r) return r;
+  // layers are independent (each has its own hidden input and output): odd
+  // layers run on the second stream with the second scratch set, forked after
+  // the ring push (motion K/V read its batch motion) and joined before the
+  // bank check (its appends change the bank length the attention reads).
+  // Profiled rounds keep one stream so that the layer events bracket layers.
+  const bool fork = !a.layer_events && ctx->side != nullptr && c.n_layers > 1;
+  if (fork && (cudaEventRecord(ctx->ev_fork, s) != cudaSuccess ||
+               cudaStreamWaitEvent(ctx->side, ctx->ev_fork, 0) != cudaSuccess))
+    return PL_ECUDA;
+  for (int l = 0; l < c.n_layers && r == PL_OK; ++l) {
+    if (a.layer_events && cudaEventRecord(a.layer_events[l], s) != cudaSuccess) {
+      r = PL_ECUDA;
+      break;
     }
-    r = single_gemm(a.hidden[l], C, w.w_qkv, 3 * C, ctx->qkv, 3 * C, static_cast<int>(M), 3 * C,
-                    C, &ctx->st->status, s);
-    if (r) return r;
-    // own K/V per frame; bank entry b of session z for the frames of session z
-    AttnSegHost segs[1 + PL_MAX_BANK];
-    segs[0] = {ctx->qkv + C, ctx->qkv + 2 * C, N, 3ll * C, static_cast<int64_t>(N) * 3 * C};
-    const int nb = ctx->have_anchors ? ctx->capacity : 1;
-    for (int b = 0; b < nb; ++b) {
-      const __half* kv = ctx->bank_kv[l] + static_cast<int64_t>(b) * N * 2 * C;
-      segs[1 + b] = {kv, kv + C, N, 2ll * C, 0};
-      if (S > 1) {
-        segs[1 + b].frame_stride = static_cast<int64_t>(ctx->capacity) * N * 2 * C;
-        segs[1 + b].n_blocks = S;
-        segs[1 + b].frame_div = 16;
-      }
-    }
-    AttnParams ap;
-    int ar = pl::attn_make_params(&ap, ctx->qkv, 3ll * C, static_cast<int64_t>(N) * 3 * C, segs,
-                                  1 + nb, F, N, H, hd, ctx->attn_o, C,
-                                  static_cast<int64_t>(N) * C);
-    if (ar) return ar == 1 ? PL_EINVAL : PL_ECUDA;
-    ap.n_fixed = 2;
-    ap.n_extra = ctx->have_anchors ? &ctx->st->appends : nullptr;
-    ap.extra_div = 16;
-    ap.extra_stride = static_cast<int>(sizeof(pl::DevState) / sizeof(int32_t));
-    ap.status = &ctx->st->status;
-    ar = pl::attn_launch(ap, hd, s);
-    if (ar) return ar == 7 ? PL_EUNSUPPORTED : PL_ECUDA;
-    uint32_t* status = &ctx->st->status;
-    const int Mi = static_cast<int>(M);
-    if (fold_layer(c, l)) {
-      // motion cross-attention, folded: per frame the scores X W_qk with the
-      // softmax over each head's 32 tokens in the GEMM epilogue (P, fp16, in
-      // the query buffer), then the block output P VM; block 2 takes block 1's
-      // output as its X
-      const int NT = 32 * H;
-      __half* P = reinterpret_cast<__half*>(ctx->qm);
-      const __half* x = ctx->attn_o;
-      const void* wq = ctx->w_oq[l];   // O (Wo Mq)
-      if (a.attn_out) {
-        // the sub-layer output is wanted: O Wo, then its motion queries
-        __half* a1 = static_cast<__half*>(a.attn_out[l]);
-        r = single_gemm(ctx->attn_o, C, w.w_o, C, a1, C, Mi, C, C, status, s);
-        if (r) return r;
-        x = a1;
-        wq = w.m_q;
-      }
-      for (int b = 0; b < ctx->motion_blocks; ++b) {
-        const bool second = b == 1;
-        __half* y = b == ctx->motion_blocks - 1 ? out : ctx->om;
-        r = from_cuda(pl::launch_motion_fold(
-            second ? ctx->motion_kv2[l] : ctx->motion_kv[l],
-            static_cast<const __half*>(second ? w.m2_q : wq),
-            static_cast<const __half*>(second ? w.m2_o : w.m_o), F, C, H, ctx->fold_wqk,
-            ctx->fold_vm, s));
-        if (r) return r;
-        r = frame_gemm(x, C, ctx->fold_wqk, NT, static_cast<int64_t>(C) * NT, P, NT, F, N, NT, C,
-                       true, status, s);
-        if (r) return r;
-        r = frame_gemm(P, NT, ctx->fold_vm, C, static_cast<int64_t>(NT) * C, y, C, F, N, C, NT,
-                       false, status, s);
-        if (r) return r;
-        x = y;
-      }
-    } else {
-      if (a.attn_out) {
-        // the sub-layer output is wanted: O Wo, then its motion queries
-        __half* a1 = static_cast<__half*>(a.attn_out[l]);
-        r = single_gemm(ctx->attn_o, C, w.w_o, C, a1, C, Mi, C, C, status, s);
-        if (r) return r;
-        r = single_gemm(a1, C, w.m_q, C, ctx->qm, C, Mi, C, C, status, s, /*out_f32=*/true);
-      } else {
-        // motion queries straight from O: O (Wo Mq)
-        r = single_gemm(ctx->attn_o, C, ctx->w_oq[l], C, ctx->qm, C, Mi, C, C, status, s,
-                        /*out_f32=*/true);
-      }
-      if (r) return r;
-      r = from_cuda(
-          pl::launch_motion_attn(ctx->qm, C, ctx->motion_kv[l], F, N, C, H, ctx->om, C, s));
-      if (r) return r;
-      if (ctx->motion_blocks == 2) {
-        // block 2's queries from block 1's output: y1 Mq2 = om (Mo Mq2)
-        if (a.attn_out) {
-          r = single_gemm(ctx->om, C, w.m_o, C, ctx->a1, C, Mi, C, C, status, s);
-          if (r) return r;
-          r = single_gemm(ctx->a1, C, w.m2_q, C, ctx->qm, C, Mi, C, C, status, s, true);
-        } else {
-          r = single_gemm(ctx->om, C, ctx->w_oq2[l], C, ctx->qm, C, Mi, C, C, status, s, true);
-        }
-        if (r) return r;
-        r = from_cuda(pl::launch_motion_attn(ctx->qm, C, ctx->motion_kv2[l], F, N, C, H, ctx->om,
-                                             C, s));
-        if (r) return r;
-      }
-      const void* w_last = ctx->motion_blocks == 2 ? w.m2_o : w.m_o;
-      r = single_gemm(ctx->om, C, w_last, C, out, C, Mi, C, C, status, s);
-      if (r) return r;
-    }
+    const bool odd = fork && (l & 1);
+    r = enqueue_layer(ctx, a, l, ctx->sc[odd ? 1 : 0], odd ? ctx->side : s);
   }
+  // the join also closes the fork after a failure, so a capture can end
+  if (fork && (cudaEventRecord(ctx->ev_join, ctx->side) != cudaSuccess ||
+               cudaStreamWaitEvent(s, ctx->ev_join, 0) != cudaSuccess))
+    return PL_ECUDA;
+  if (r) return r;
   if (a.layer_events && c.n_layers > 0 &&
       cudaEventRecord(a.layer_events[c.n_layers], s) != cudaSuccess)
     return PL_ECUDA;
@@ -850,6 +891,13 @@ pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_
     delete ctx;
     return PL_ECUDA;
   }
+  // the round's second stream (odd layers) and its fork / join events
+  if (cudaStreamCreateWithFlags(&ctx->side, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ctx->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ctx->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+    pl_ctx_destroy(ctx);
+    return PL_ECUDA;
+  }
   {
     const char* prof = std::getenv("PL_PROFILE");
     ctx->profile = prof && prof[0] == '1';
@@ -873,6 +921,12 @@ pl_status pl_ctx_destroy(pl_ctx* ctx) {
     if (ctx->ev_free[b]) cudaEventDestroy(ctx->ev_free[b]);
   }
   if (ctx->copy_stream) cudaStreamDestroy(ctx->copy_stream);
+  if (ctx->side) {
+    cudaStreamSynchronize(ctx->side);
+    cudaStreamDestroy(ctx->side);
+  }
+  if (ctx->ev_fork) cudaEventDestroy(ctx->ev_fork);
+  if (ctx->ev_join) cudaEventDestroy(ctx->ev_join);
   for (auto& e : ctx->prof_ev)
     if (e) cudaEventDestroy(e);
   delete ctx;
