@@ -88,6 +88,14 @@ int device_sms() {
 
 // ====================================================================== context
 
+// streams one round's layers are spread over (inside its captured graph).
+// Measured on the 512x512 round (same box, three runs each): one stream
+// 19.68-19.87 ms, two 19.38-19.49 ms, three 19.34-19.44 ms, four 19.25-19.37
+// ms; each stream beyond the first holds its own layer scratch (~340 MB per
+// session at 512x512), so two.
+constexpr int kRoundStreams = 2;
+static_assert(kRoundStreams >= 2, "the fork and join expect a second stream");
+
 struct pl_ctx {
   pl_config cfg;
   int sessions;        // S independent streams; per-stream buffers are [S][...]
@@ -106,9 +114,9 @@ struct pl_ctx {
   float* motion_kv2[PL_MAX_LAYERS];  // second motion block's, as motion_kv
   __half* w_oq[PL_MAX_LAYERS];        // fp16 [C][C] = Wo Mq
   __half* w_oq2[PL_MAX_LAYERS];       // fp16 [C][C] = Mo Mq2 (two motion blocks)
-  // per-layer scratch, two sets: the round runs even layers on its stream
-  // with set 0 and odd layers on a second stream with set 1 (the layers are
-  // independent: each has its own hidden input and output)
+  // per-layer scratch, one set per round stream: layer l runs on stream
+  // l % kRoundStreams with set l % kRoundStreams (the layers are independent:
+  // each has its own hidden input and output)
   struct Scratch {
     __half* qkv;
     __half* attn_o;
@@ -119,9 +127,10 @@ struct pl_ctx {
     __half* out_default;
     __half* fold_wqk;   // folded motion path: fp16 [S][16][C][32 H]
     __half* fold_vm;    // and fp16 [S][16][32 H][C]
-  } sc[2];
-  cudaStream_t side;               // the round's second stream (odd layers)
-  cudaEvent_t ev_fork, ev_join;    // its fork after the ring push, its join
+  } sc[kRoundStreams];
+  cudaStream_t side[kRoundStreams - 1];   // the round's other streams
+  cudaEvent_t ev_fork;                    // their fork after the ring push
+  cudaEvent_t ev_join[kRoundStreams - 1];  // and their joins
   pl::DdimCoef coef;
   bool initialised;
   bool have_anchors;
@@ -204,7 +213,7 @@ size_t layout(const pl_config& c, pl_ctx* ctx) {
   for (int l = 0; l < c.n_layers; ++l)
     if (fold_layer(c, l) && c.layer_channels[l] > fold_c) fold_c = c.layer_channels[l];
   const int64_t fold_elems = S * 16 * fold_c * 32 * c.heads;
-  for (int k = 0; k < 2; ++k) {
+  for (int k = 0; k < kRoundStreams; ++k) {
     uint8_t* qkv = take(sizeof(__half) * 3 * max_nc);
     uint8_t* ao = take(sizeof(__half) * max_nc);
     uint8_t* a1 = take(sizeof(__half) * max_nc);
@@ -466,27 +475,33 @@ pl_status enqueue_round(pl_ctx* ctx, const RoundArgs& a, cudaStream_t s) {
                                                ctx->batch_motion, a.new_noise, a.new_motion,
                                                ctx->frame_elems, S, s));
   if (r) return r;
-  // layers are independent (each has its own hidden input and output): odd
-  // layers run on the second stream with the second scratch set, forked after
-  // the ring push (motion K/V read its batch motion) and joined before the
-  // bank check (its appends change the bank length the attention reads).
-  // Profiled rounds keep one stream so that the layer events bracket layers.
-  const bool fork = !a.layer_events && ctx->side != nullptr && c.n_layers > 1;
-  if (fork && (cudaEventRecord(ctx->ev_fork, s) != cudaSuccess ||
-               cudaStreamWaitEvent(ctx->side, ctx->ev_fork, 0) != cudaSuccess))
-    return PL_ECUDA;
+  // layers are independent (each has its own hidden input and output):
+  // layer l runs on round stream l % kRoundStreams with its scratch set, the
+  // other streams forked after the ring push (motion K/V read its batch
+  // motion) and joined before the DDIM step and the bank check (its appends
+  // change the bank length the attention reads). Profiled rounds keep one
+  // stream so that the layer events bracket layers.
+  const bool fork = !a.layer_events && kRoundStreams > 1 && ctx->side[0] != nullptr &&
+                    c.n_layers > 1;
+  if (fork) {
+    if (cudaEventRecord(ctx->ev_fork, s) != cudaSuccess) return PL_ECUDA;
+    for (int k = 0; k + 1 < kRoundStreams; ++k)
+      if (cudaStreamWaitEvent(ctx->side[k], ctx->ev_fork, 0) != cudaSuccess) return PL_ECUDA;
+  }
   for (int l = 0; l < c.n_layers && r == PL_OK; ++l) {
     if (a.layer_events && cudaEventRecord(a.layer_events[l], s) != cudaSuccess) {
       r = PL_ECUDA;
       break;
     }
-    const bool odd = fork && (l & 1);
-    r = enqueue_layer(ctx, a, l, ctx->sc[odd ? 1 : 0], odd ? ctx->side : s);
+    const int k = fork ? l % kRoundStreams : 0;
+    r = enqueue_layer(ctx, a, l, ctx->sc[k], k ? ctx->side[k - 1] : s);
   }
-  // the join also closes the fork after a failure, so a capture can end
-  if (fork && (cudaEventRecord(ctx->ev_join, ctx->side) != cudaSuccess ||
-               cudaStreamWaitEvent(s, ctx->ev_join, 0) != cudaSuccess))
-    return PL_ECUDA;
+  // the joins also close the fork after a failure, so a capture can end
+  if (fork)
+    for (int k = 0; k + 1 < kRoundStreams; ++k)
+      if (cudaEventRecord(ctx->ev_join[k], ctx->side[k]) != cudaSuccess ||
+          cudaStreamWaitEvent(s, ctx->ev_join[k], 0) != cudaSuccess)
+        return PL_ECUDA;
   if (r) return r;
   if (a.layer_events && c.n_layers > 0 &&
       cudaEventRecord(a.layer_events[c.n_layers], s) != cudaSuccess)
@@ -891,10 +906,12 @@ pl_status pl_ctx_create(const pl_config* cfg, void* workspace, size_t workspace_
     delete ctx;
     return PL_ECUDA;
   }
-  // the round's second stream (odd layers) and its fork / join events
-  if (cudaStreamCreateWithFlags(&ctx->side, cudaStreamNonBlocking) != cudaSuccess ||
-      cudaEventCreateWithFlags(&ctx->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&ctx->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+  // the round's other streams and their fork / join events
+  bool made = cudaEventCreateWithFlags(&ctx->ev_fork, cudaEventDisableTiming) == cudaSuccess;
+  for (int k = 0; made && k + 1 < kRoundStreams; ++k)
+    made = cudaStreamCreateWithFlags(&ctx->side[k], cudaStreamNonBlocking) == cudaSuccess &&
+           cudaEventCreateWithFlags(&ctx->ev_join[k], cudaEventDisableTiming) == cudaSuccess;
+  if (!made) {
     pl_ctx_destroy(ctx);
     return PL_ECUDA;
   }
@@ -921,12 +938,14 @@ pl_status pl_ctx_destroy(pl_ctx* ctx) {
     if (ctx->ev_free[b]) cudaEventDestroy(ctx->ev_free[b]);
   }
   if (ctx->copy_stream) cudaStreamDestroy(ctx->copy_stream);
-  if (ctx->side) {
-    cudaStreamSynchronize(ctx->side);
-    cudaStreamDestroy(ctx->side);
+  for (int k = 0; k + 1 < kRoundStreams; ++k) {
+    if (ctx->side[k]) {
+      cudaStreamSynchronize(ctx->side[k]);
+      cudaStreamDestroy(ctx->side[k]);
+    }
+    if (ctx->ev_join[k]) cudaEventDestroy(ctx->ev_join[k]);
   }
   if (ctx->ev_fork) cudaEventDestroy(ctx->ev_fork);
-  if (ctx->ev_join) cudaEventDestroy(ctx->ev_join);
   for (auto& e : ctx->prof_ev)
     if (e) cudaEventDestroy(e);
   delete ctx;
