@@ -509,8 +509,13 @@ pl_status pl_ctx_bank_check(pl_ctx* ctx, const float* queries, int n_queries,
  * when given, each layer's reference-attention sub-layer output (before the
  * motion cross-attention) is written there, and the round then applies Wo
  * and Mq (and Mo, Mq2) as separate projections instead of their products.
+ * Layers of 1024 tokens per frame and more evaluate the motion
+ * cross-attention per head as scores x (Mq K^T / sqrt(hd)) and output
+ * P (V Mo) (the same function; fp16 roundings of those products).
  * The round is recorded as a CUDA graph on the first call and replayed while
- * the pointer arguments stay the same. */
+ * the pointer arguments stay the same; inside the graph the layers run on
+ * two streams the context owns, forked from and joined back into `stream`,
+ * so the whole round is ordered on `stream` like any other call. */
 pl_status pl_stream_round(pl_ctx* ctx, const float* new_noise, const float* new_motion,
                           const void* const* hidden, const float* eps, float* out_frames,
                           uint8_t* appended, void* const* layer_out,
